@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the NOSA decode step on B200 (one JSON line on rank 0).
+
+Workload (default): offloaded batch decode at B=64 -- 32 query / 8 KV heads,
+head_dim 128, 4096-token context (64 blocks of 64), budget 16 blocks (12
+query-aware + 4 agnostic, overlap >= 13), full KV in pinned host memory, GPU
+block cache of 32 blocks per (sequence, KV head), AR(1) queries rho = 0.95.
+
+A step is one pass of the whole path: score -> select -> fetch (plan + PCIe
+gather of the misses) -> sparse attention, captured once in a CUDA graph and
+replayed.  Step 0 (cold cache) and the other warm-up steps run eagerly and are
+not timed.  The per-step traffic (256 MiB of selected K/V + 32 MiB of pooled
+keys) exceeds the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME]
+
+Under torchrun every rank runs its own copy of the workload on its own GPU
+(weak scaling, no collective on the data path); rank 0 prints the line with
+the max-over-ranks time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NOSA decode tokens/s at B=64 (1 GPU); HBM & PCIe GB/s vs roofline"
+UNIT = "tokens/s"
+HBM_NOMINAL_GBS = 8000.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=8)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="offload_b64")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=50)
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        return {}
+
+
+def hbm_bytes_per_step(w, fetched_blocks_per_step):
+    """Algorithmic HBM bytes of one step: pooled keys, scores (fp64 write +
+    read), agnostic scores, selected K+V, cache writes of fetched blocks, q and
+    out."""
+    U, n, R, d = w.units, w.n_blocks0, w.block // w.sub_block, w.head_dim
+    pooled = U * n * R * d * 2
+    scores = U * n * 8 * 2
+    agn = U * n * 4
+    selected = U * w.k * w.block * d * 2 * 2
+    writes = fetched_blocks_per_step * w.block * d * 2 * 2
+    qo = w.batch * w.n_q_heads * d * 2 * 2
+    return pooled + scores + agn + selected + writes + qo
+
+
+def measure_h2d_peak(torch, dev, mib=256, reps=3):
+    """Copy-engine host->device bandwidth from pinned memory (GB/s)."""
+    n = mib * (1 << 20)
+    src = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(n, dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream(dev)
+    best = 0.0
+    with torch.cuda.stream(s):
+        for _ in range(reps + 1):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            dst.copy_(src, non_blocking=True)
+            e1.record(s)
+            s.synchronize()
+            best = max(best, n / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del src, dst
+    return best
+
+
+def cpu_baseline(w, target_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the workload on the
+    host cores (OpenMP over units).  Returns (tokens/s, cores, sample text)."""
+    import numpy as np
+    import oracle
+    from kv_cache_decode_step_b200 import inputs
+
+    def run(n_units, steps):
+        units = list(range(n_units))
+        d = inputs.generate(w.with_(steps=steps), units=units)
+        cfg = oracle.cfg_from_workload(w, steps=steps)
+        t0 = time.perf_counter()
+        _, _, _, th = oracle.run_units(cfg, d["k"], d["v"], d["a"], d["q"], attend_steps=None)
+        return time.perf_counter() - t0, th
+
+    t_probe, th = run(min(w.units, 16), 2)
+    per_unit_step = t_probe / (min(w.units, 16) * 2)
+    n_units = min(w.units, 64)
+    steps = max(2, min(64, int(target_s / max(per_unit_step * n_units, 1e-6))))
+    t, th = run(n_units, steps)
+    step_time = t / steps * (w.units / n_units)
+    return (w.batch / step_time, th,
+            f"oracle on {n_units} of {w.units} units x {steps} steps (all phases, attention every "
+            f"step), scaled to the full batch; {t:.1f} s of CPU work")
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    from kv_cache_decode_step_b200 import configs
+    import oracle
+    from kv_cache_decode_step_b200 import inputs
+    w = configs.get(args.workload)
+    # bounded sample per step: a few units of the workload, scaled to the batch
+    n_units = min(w.units, 16)
+    steps = args.warmup + args.steps
+    d = inputs.generate(w.with_(steps=max(steps, 2)), units=list(range(n_units)))
+    cfg = oracle.cfg_from_workload(w, steps=max(steps, 2))
+    t0 = time.perf_counter()
+    _, _, _, th = oracle.run_units(cfg, d["k"], d["v"], d["a"], d["q"], attend_steps=None)
+    t = time.perf_counter() - t0
+    step_time = t / max(steps, 2) * (w.units / n_units)
+    value = w.batch / step_time
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_time * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "context": w.context, "k": w.k,
+                   "k_query": w.k_query, "k_agnostic": w.k_agnostic, "min_overlap": w.min_overlap,
+                   "cache_slots": w.cache_slots, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": th, "kind": "oracle",
+                         "sample": f"fp64 CPU oracle on {n_units} of {w.units} units x {max(steps, 2)} "
+                                   f"steps, scaled to the full batch"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from kv_cache_decode_step_b200 import build, configs, inputs, nosa, runner
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    build.build()
+
+    base = configs.get(args.workload)
+    total = 1 + args.warmup + args.steps + args.e2e_steps + 64
+    w = base.with_(steps=max(base.steps, total))
+    data = inputs.generate(w)
+    dec = runner.Decoder(w, data, device=local)
+
+    h2d_peak = measure_h2d_peak(torch, dev)
+
+    # warm-up: step 0 (cold cache) plus W eager steps
+    for _ in range(1 + args.warmup):
+        dec.step()
+    dec.stream.synchronize()
+    dec.capture()
+    dec.replay()  # one untimed replay
+    dec.stream.synchronize()
+    nosa.nosa_reset_stats(dec.ctx, dec.stream)
+
+    # ---- timed region: K graph replays
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(dec.stream)
+    for _ in range(args.steps):
+        dec.replay()
+    e1.record(dec.stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    st = dec.stats()
+    dec.check()
+    t_max = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    ms_max = float(t_max.item())
+    ms_step = ms_max / args.steps
+    value = world * w.batch * args.steps / (ms_max * 1e-3)
+
+    fetched_blocks = st["misses"] / args.steps
+    pcie_bytes = st["fetched_bytes"] / args.steps
+    hbm_bytes = hbm_bytes_per_step(w, fetched_blocks)
+    peaks = measured_peaks()
+    hbm_meas = float(peaks.get("hbm_gbs", 6650.0))
+    hbm_src = "of measured" if "hbm_gbs" in peaks else "of fallback"
+    t_hbm = hbm_bytes / (HBM_NOMINAL_GBS * 1e9)
+    t_hbm_meas = hbm_bytes / (hbm_meas * 1e9)
+    t_pcie = pcie_bytes / (h2d_peak * 1e9)
+    step_s = ms_step * 1e-3
+
+    # ---- instrumented pass: same graph, per-phase events per step
+    phase = instrumented_pass(torch, dec, w, nosa, n=min(args.steps, 50))
+
+    # ---- end to end through host buffers: q from pinned host, out to pinned host
+    e2e = e2e_pass(torch, dec, w, nosa, args.e2e_steps)
+
+    launches_per_step = 8  # score, select, plan, gather, attend x2, combine, advance
+    gather_ms = phase["gather_ms"]
+    attn_ms = phase["decode_ms"]
+    gather_gbs = (phase["fetched_bytes_per_step"] / (gather_ms * 1e-3) / 1e9) if gather_ms > 0 else 0.0
+    attn_bytes = w.units * w.k * w.block * w.head_dim * 2 * 2 + w.batch * w.n_q_heads * w.head_dim * 2 * 2
+    attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9 if attn_ms > 0 else 0.0
+    rl_gather = {"kernel": "gather_kernel", "bound": "pcie", "achieved": gather_gbs, "peak": h2d_peak,
+                 "unit": "GB/s", "frac": gather_gbs / h2d_peak if h2d_peak else None, "traffic": None,
+                 "peak_source": "pinned cudaMemcpyAsync H2D measured in this run (256 MiB)",
+                 "bytes_per_launch": phase["fetched_bytes_per_step"], "ms_per_launch": gather_ms}
+    rl_attn = {"kernel": "decode_kernel+combine_kernel", "bound": "hbm", "achieved": attn_gbs,
+               "peak": hbm_meas, "unit": "GB/s", "frac": attn_gbs / hbm_meas, "traffic": None,
+               "peak_source": f"hbm_gbs {hbm_src}", "bytes_per_launch": attn_bytes, "ms_per_launch": attn_ms}
+    dominant, other = (rl_gather, rl_attn) if gather_ms >= attn_ms else (rl_attn, rl_gather)
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            v, cores, sample = cpu_baseline(w)
+            cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 K/V, U(0,1) agnostic scores, AR(1) queries)",
+            "config": {"workload": w.name, "batch": w.batch, "context": w.context,
+                       "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                       "block": w.block, "sub_block": w.sub_block, "k": w.k, "k_query": w.k_query,
+                       "k_agnostic": w.k_agnostic, "min_overlap": w.min_overlap,
+                       "cache_slots": w.cache_slots, "kv": "pinned host", "parallelism": f"replicas x{world}",
+                       "l2": "per-step traffic 288 MiB > 126 MB L2, no flush", "graph": "cuda graph replay"},
+            "roofline": dominant,
+            "roofline_other": other,
+            "roofline_step": {
+                "hbm_bytes_per_step": hbm_bytes, "pcie_bytes_per_step": pcie_bytes,
+                "h2d_peak_gbs": h2d_peak, "t_hbm_nominal_us": t_hbm * 1e6, "t_hbm_measured_us": t_hbm_meas * 1e6,
+                "t_pcie_us": t_pcie * 1e6,
+                "frac_nominal": max(t_hbm, t_pcie) / step_s,
+                "frac_measured": max(t_hbm_meas, t_pcie) / step_s,
+                "hbm_gbs_achieved": hbm_bytes / step_s / 1e9, "h2d_gbs_achieved": pcie_bytes / step_s / 1e9,
+            },
+            "decode_stats": {
+                "hit_rate": st["hits"] / max(1, st["hits"] + st["misses"]),
+                "fetched_blocks_per_step": fetched_blocks,
+                "fetched_mib_per_step": pcie_bytes / 2**20,
+                "locality_mean": st["overlap_sum"] / max(1, st["overlap_terms"] * w.k),
+                "locality_min": st["min_overlap"] / w.k,
+            },
+            "phases_ms": phase,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(result), flush=True)
+    dec.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def instrumented_pass(torch, dec, w, nosa, n):
+    """Replay the same step n times with events between the ABI calls (eager
+    issue on the same streams) and read per-phase durations after each step."""
+    s, cs = dec.stream, dec.copy_stream
+    ev = {k: torch.cuda.Event(enable_timing=True) for k in ("a", "b", "c", "d", "g", "e")}
+    acc = {"score_ms": 0.0, "select_ms": 0.0, "plan_ms": 0.0, "gather_ms": 0.0, "decode_ms": 0.0, "step_ms": 0.0}
+    misses0 = dec.stats()["fetched_bytes"]
+    for _ in range(n):
+        t = dec.t
+        with torch.cuda.stream(s):
+            dec.q.copy_(dec.q_all[t], non_blocking=True)
+            ev["a"].record(s)
+            nosa.nosa_score_blocks(dec.ctx, dec.q, dec.scores, s)
+            ev["b"].record(s)
+            nosa.nosa_select(dec.ctx, dec.scores, dec.sel, s)
+            ev["c"].record(s)
+            nosa.nosa_fetch_missing(dec.ctx, dec.sel, dec.fetch, dec.n_fetch, s, cs)
+            ev["d"].record(s)
+            ev["g"].record(cs)
+            nosa.nosa_sparse_decode(dec.ctx, dec.q, dec.sel, dec.out, s)
+            ev["e"].record(s)
+        dec.t += 1
+        torch.cuda.synchronize()
+        acc["score_ms"] += ev["a"].elapsed_time(ev["b"])
+        acc["select_ms"] += ev["b"].elapsed_time(ev["c"])
+        acc["plan_ms"] += ev["c"].elapsed_time(ev["d"])
+        acc["gather_ms"] += ev["d"].elapsed_time(ev["g"])
+        acc["decode_ms"] += ev["d"].elapsed_time(ev["e"])
+        acc["step_ms"] += ev["a"].elapsed_time(ev["e"])
+    out = {k: v / n for k, v in acc.items()}
+    out["fetched_bytes_per_step"] = (dec.stats()["fetched_bytes"] - misses0) / n
+    out["steps"] = n
+    out["note"] = ("decode_ms spans attention over hits (overlapping the gather), the wait for the "
+                   "gather, attention over misses, combine and step advance")
+    return out
+
+
+def e2e_pass(torch, dec, w, nosa, n):
+    """End to end through the binding: every step copies q from pinned host
+    memory, runs the four calls and reads the output back to pinned host memory."""
+    q_host = dec.q_all[:].cpu().pin_memory()
+    out_host = torch.empty_like(dec.out, device="cpu").pin_memory()
+    s = dec.stream
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    t0 = time.perf_counter()
+    for _ in range(n):
+        t = dec.t
+        with torch.cuda.stream(s):
+            dec.q.copy_(q_host[t], non_blocking=True)
+            dec._calls(None)
+            out_host.copy_(dec.out, non_blocking=True)
+        s.synchronize()
+        dec.t += 1
+    e1.record(s)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    ms = e0.elapsed_time(e1)
+    qb = dec.q.numel() * 2
+    ob = dec.out.numel() * 2
+    return {"value": w.batch * n / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": qb,
+            "d2h_bytes_per_step": ob, "steps": n, "wall_tokens_per_s": w.batch * n / wall,
+            "note": "eager ABI calls, q H2D and out D2H inside the timed region, host sync per step"}
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

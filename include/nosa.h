@@ -1,0 +1,232 @@
+/*
+ * nosa.h -- C ABI of libnosa.so: the NOSA decode step on one B200 (sm_100a).
+ *
+ * NOSA (NOSA: Native and Offloadable Sparse Attention, paperlayer summary,
+ * App. A) decodes each step as: select blocks -> move the cache-missed KV
+ * blocks CPU -> GPU -> attend with the GPU-resident blocks.  This library
+ * splits that step into four calls, made in this order once per step:
+ *
+ *   nosa_score_blocks   block scores from pooled keys        (§3.1)
+ *   nosa_select         eviction-bounded query-agnostic set + capped
+ *                       query-aware top-k, overlap >= m       (§3.1, App. E)
+ *   nosa_fetch_missing  set difference against the GPU block cache and a
+ *                       zero-copy gather of the misses over PCIe (§4)
+ *   nosa_sparse_decode  GQA attention over the selected blocks (App. A)
+ *
+ * plus nosa_append_token first when the sequence grows during decoding.
+ *
+ * Terms.  A unit is one (sequence b, KV head g), numbered u = b*n_kv_heads + g.
+ * G = n_q_heads / n_kv_heads query heads share a KV head; query head h uses KV
+ * head h / G.  A block is P = 64 tokens, a sub-block Q = 16 tokens, R = P/Q = 4
+ * sub-blocks per block, head_dim d = 128.  n is the number of closed (full)
+ * blocks of every unit; a partially filled last block (the tail) is attended
+ * but never scored, selected or fetched.  k = k_query + k_agnostic.
+ *
+ * Conventions (every entry point):
+ *  - Returns a nosa_status and never aborts, throws or exits.  On failure,
+ *    nosa_last_error() gives a message for the calling thread.
+ *  - "device" buffers are CUDA device memory of the context's device; "host"
+ *    buffers are ordinary host memory; "pinned host" buffers are page-locked
+ *    (cudaHostAlloc / cudaHostRegister) and therefore device-addressable.
+ *  - Every buffer is owned by the caller, who keeps it alive and unmodified
+ *    until the work queued on the stream that reads it has finished.
+ *  - Calls are asynchronous on the given stream unless marked "synchronous".
+ *    A CUDA error raised by earlier work may surface in a later call as
+ *    NOSA_ERR_CUDA.  The step calls enqueue work only; they are safe to
+ *    capture in a CUDA graph, and every per-step quantity (step counter, block
+ *    count, tail length) lives in device memory so that replays advance it.
+ *  - Out-of-order step calls return NOSA_ERR_ORDER and enqueue nothing.
+ *  - A context is not thread-safe; use one context per thread or serialise.
+ *  - Device-side waits are bounded (about 1 s).  A wait that runs out sets an
+ *    error bit that nosa_check_errors() reports as NOSA_ERR_TIMEOUT.
+ */
+#ifndef NOSA_H
+#define NOSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NOSA_API __attribute__((visibility("default")))
+#else
+#define NOSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA header.
+ * NULL means the legacy default stream. */
+typedef struct CUstream_st* nosa_stream_t;
+
+typedef enum {
+  NOSA_OK = 0,
+  NOSA_ERR_INVALID = -1,        /* bad argument, config or pointer kind */
+  NOSA_ERR_CUDA = -2,           /* a CUDA runtime/driver call failed */
+  NOSA_ERR_NOMEM = -3,          /* device allocation failed */
+  NOSA_ERR_ORDER = -4,          /* step calls out of order */
+  NOSA_ERR_TIMEOUT = -5,        /* a bounded device-side wait ran out */
+  NOSA_ERR_UNIMPLEMENTED = -6   /* configuration outside what v1 supports */
+} nosa_status;
+
+typedef struct nosa_ctx nosa_ctx;
+
+/* Shape and budget of a decode batch.  v1 supports head_dim = 128, block = 64,
+ * sub_block = 16 and 1 <= G <= 8 (otherwise NOSA_ERR_UNIMPLEMENTED). */
+typedef struct {
+  int batch;          /* B >= 1 sequences */
+  int n_q_heads;      /* H_q, a multiple of n_kv_heads */
+  int n_kv_heads;     /* H_kv >= 1 */
+  int head_dim;       /* d, must be 128 */
+  int block;          /* P, must be 64 */
+  int sub_block;      /* Q, must be 16 */
+  int k_query;        /* k_q >= 0 query-aware blocks per unit and step */
+  int k_agnostic;     /* k_e >= 0 query-agnostic blocks per unit and step */
+  int min_overlap;    /* m = ceil(gamma0 * k), 0 <= m <= k: at least m blocks
+                         of S(t) were also in S(t-1) (NOSA summary §3.1) */
+  int max_blocks;     /* block capacity per unit (prompt + growth), >= k, <= 8192 */
+  int cache_slots;    /* 0: KV resident in HBM; else GPU cache blocks per unit,
+                         k <= cache_slots <= 1024, KV in pinned host memory */
+} nosa_config;
+
+/* Running totals since the last attach or nosa_reset_stats. */
+typedef struct {
+  int64_t steps;           /* decode steps completed (nosa_sparse_decode calls) */
+  int64_t selected;        /* sum over units and steps of |S(t)| */
+  int64_t hits;            /* selected blocks already in the GPU cache */
+  int64_t misses;          /* selected blocks fetched over PCIe */
+  int64_t fetched_bytes;   /* K+V bytes moved host -> device by the gather */
+  int64_t overlap_sum;     /* sum over units, steps t >= 1 of |S(t) ∩ S(t-1)| */
+  int64_t overlap_terms;   /* number of (unit, step >= 1) terms in overlap_sum */
+  int32_t min_overlap;     /* min over units, steps t >= 1 of |S(t) ∩ S(t-1)|
+                              (INT32_MAX before step 1) */
+  int32_t max_fetch;       /* max over units, steps t >= 1 of blocks fetched */
+  uint32_t error_bits;     /* device error bits (see nosa_check_errors) */
+  int32_t n_closed;        /* closed blocks per unit now */
+  int32_t tail_len;        /* tokens in the open tail block now */
+  int32_t reserved;
+} nosa_stats;
+
+/* Validate cfg and allocate the context's device state on the current device:
+ * pooled keys bf16 [U, max_blocks*R, d], agnostic scores fp32 [U, max_blocks],
+ * selection state, the GPU block cache bf16 [U, cache_slots, P, d] x 2 (K, V)
+ * with its tables, the open tail block bf16 [U, P, d] x 2 and attention
+ * partials.  Synchronous.  *out is set only on NOSA_OK. */
+NOSA_API nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out);
+
+/* Free everything nosa_create allocated (synchronises the device first).
+ * NULL is ignored. */
+NOSA_API void nosa_destroy(nosa_ctx* ctx);
+
+/* Attach the KV of every unit and reset the decode state (step 0, cold cache).
+ * k, v: bf16 [U, max_blocks*P, d] row-major (unit, token, dim).  With
+ *   cache_slots > 0 they must be pinned host memory: the full cache lives on the
+ *   host (NOSA summary §1, §4) and blocks closed during decoding are written
+ *   through into it.  With cache_slots = 0 they are device memory.
+ *   Base addresses must be 16-byte aligned.
+ * n_tokens: prompt tokens per unit, k*P <= n_tokens <= max_blocks*P.  Tokens
+ *   beyond the last full block become the open tail block.
+ * agnostic: device fp32 [U, max_blocks], the query-agnostic score of every
+ *   block (copied; entries of blocks that close later are replaced by
+ *   nosa_append_token's value).
+ * Builds the pooled keys (one read of K; over PCIe when offloaded) on stream.
+ */
+NOSA_API nosa_status nosa_attach_kv(nosa_ctx* ctx, const void* k, const void* v, int n_tokens,
+                           const float* agnostic, nosa_stream_t stream);
+
+/* Append one token per unit to the open tail block (first call of a step).
+ * k_new, v_new: device bf16 [B, H_kv, d].  agnostic_if_close: device fp32 [U]
+ * or NULL; it becomes the agnostic score of the tail block if this token fills
+ * it, in which case nosa_sparse_decode closes the block at the end of the step
+ * (pooled keys built, written through to the host KV, candidate from the next
+ * step on).  NOSA_ERR_INVALID when the unit would exceed max_blocks*P tokens. */
+NOSA_API nosa_status nosa_append_token(nosa_ctx* ctx, const void* k_new, const void* v_new,
+                              const float* agnostic_if_close, nosa_stream_t stream);
+
+/* Two-stage block scores (NOSA summary §3.1): for each unit and closed block j,
+ *   scores[u*max_blocks + j] = max_{r<R} sum_{h in group(u)} q_h . kbar[u, j*R + r]
+ * where kbar is the mean of each sub-block's 16 keys rounded once to bf16.
+ * Products are exact and sums are fp64.  q: device bf16 [B, H_q, d].
+ * scores: device fp64 [U, max_blocks]; entries j >= n are left untouched. */
+NOSA_API nosa_status nosa_score_blocks(nosa_ctx* ctx, const void* q, double* scores, nosa_stream_t stream);
+
+/* Selection (NOSA summary §2.1, §3.1, App. E), per unit:
+ *   Gamma_e(t) = top-k_e by agnostic score of Gamma_e(t-1) plus the blocks
+ *                closed since the last step (all closed blocks at step 0);
+ *                an evicted block never re-enters Gamma_e.
+ *   c_t        = max(0, (k - m) - |Gamma_e(t) \ S(t-1)|)   (no cap at step 0)
+ *   Gamma_q(t) = top-k_q by score of (S(t-1) \ Gamma_e(t)) ∪ top-c_t of the
+ *                blocks in neither Gamma_e(t) nor S(t-1)
+ *   S(t)       = Gamma_e(t) ∪ Gamma_q(t)
+ * Ties go to the lower block id.  scores: device fp64 as written by
+ * nosa_score_blocks.  sel: device int32 [U, k], S(t) ascending, -1 padded. */
+NOSA_API nosa_status nosa_select(nosa_ctx* ctx, const double* scores, int32_t* sel, nosa_stream_t stream);
+
+/* Cache planning and miss gather (NOSA summary §4, App. A).  Per unit the
+ * misses M = S(t) \ R(t-1) (R = blocks resident in the GPU cache) get slots:
+ * free slots first (lowest first), then resident blocks outside S(t), least
+ * recently selected first, lower block id on ties.  Only blocks unused by this
+ * step are replaced.  The K and V of each miss (2 x 16 KiB) are then copied
+ * from pinned host memory into its slot by a zero-copy gather kernel.
+ * sel: device int32 [U, k] from nosa_select.  fetch: device int32 [U, k], the
+ * missed block ids ascending, -1 padded.  n_fetch: device int32 [U].
+ * Planning runs on compute; the gather on copy, which may equal compute.  A
+ * separate copy stream lets nosa_sparse_decode attend to the hit blocks while
+ * the misses are in flight.  With KV resident (cache_slots = 0) nothing is
+ * copied: fetch is all -1 and n_fetch all 0. */
+NOSA_API nosa_status nosa_fetch_missing(nosa_ctx* ctx, const int32_t* sel, int32_t* fetch,
+                               int32_t* n_fetch, nosa_stream_t compute, nosa_stream_t copy);
+
+/* Block-sparse GQA attention (NOSA summary App. A): for each query head h of
+ * unit u,  out_h = sum_t softmax_t(q_h . K_t / sqrt(d)) V_t  over the tokens of
+ * the selected blocks plus the open tail, in fp32 with bf16 inputs; written as
+ * bf16.  q: device bf16 [B, H_q, d]; sel: the same buffer passed to
+ * nosa_select; out: device bf16 [B, H_q, d].  Ends the step: closes a full
+ * tail block and advances the step counter. */
+NOSA_API nosa_status nosa_sparse_decode(nosa_ctx* ctx, const void* q, const int32_t* sel, void* out,
+                               nosa_stream_t stream);
+
+/* Synchronous.  Copies the running totals into *stats. */
+NOSA_API nosa_status nosa_get_stats(nosa_ctx* ctx, nosa_stats* stats);
+
+/* Zero the running totals (asynchronous on stream). */
+NOSA_API nosa_status nosa_reset_stats(nosa_ctx* ctx, nosa_stream_t stream);
+
+/* Synchronous.  NOSA_ERR_TIMEOUT if a bounded device wait ran out,
+ * NOSA_ERR_INVALID if a device-side bounds or capacity check fired, else
+ * NOSA_OK.  Bits: 1 wait timeout, 2 append beyond capacity, 4 cache planning
+ * found no slot, 8 gather or decode index out of range. */
+NOSA_API nosa_status nosa_check_errors(nosa_ctx* ctx);
+
+/* Synchronous.  Host int32 [U, cache_slots]: the block held by each cache
+ * slot, -1 if free.  NOSA_ERR_INVALID when KV is resident. */
+NOSA_API nosa_status nosa_read_cache_map(nosa_ctx* ctx, int32_t* slot_block);
+
+/* Synchronous checkpoint of the decode state: step counter, block count,
+ * Gamma_e, S(t-1), cache tables, agnostic scores and the open tail block.
+ * Pass buf = NULL to query the size in *size.  Cache contents and pooled keys
+ * are not stored: nosa_set_state rebuilds them from the attached KV. */
+NOSA_API nosa_status nosa_get_state(nosa_ctx* ctx, void* buf, size_t* size);
+
+/* Synchronous restore of a nosa_get_state blob taken from a context with the
+ * same config and attached KV.  Rebuilds pooled keys and refills the cache. */
+NOSA_API nosa_status nosa_set_state(nosa_ctx* ctx, const void* buf, size_t size);
+
+/* Diagnostic: enqueue a kernel that waits until *flag (device or pinned host
+ * int32) becomes nonzero or timeout_ms elapses; on timeout it sets error bit 1
+ * and returns, leaving the context usable. */
+NOSA_API nosa_status nosa_debug_wait_flag(nosa_ctx* ctx, const int32_t* flag, int timeout_ms,
+                                 nosa_stream_t stream);
+
+/* Message of the last failure on the calling thread ("" if none). */
+NOSA_API const char* nosa_last_error(void);
+
+/* Library version string. */
+NOSA_API const char* nosa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NOSA_H */

@@ -1,0 +1,293 @@
+// nosa_internal.cuh -- device-side state, kernel parameter blocks and inline PTX
+// shared by the kernels of libnosa.so.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nosa {
+
+constexpr int kD = 128;     // head dim
+constexpr int kP = 64;      // tokens per block
+constexpr int kQ = 16;      // tokens per sub-block
+constexpr int kR = kP / kQ; // sub-blocks per block
+constexpr int kMaxG = 8;    // query heads per KV head (mma N = 8)
+constexpr int kRowU4 = kD * 2 / 16;  // 16-byte words per token row (16)
+constexpr int kBlockBytes = kP * kD * 2;  // 16 KiB: one block of K (or of V)
+
+enum : unsigned {
+  ERR_TIMEOUT = 1u,
+  ERR_CAPACITY = 2u,
+  ERR_NOSLOT = 4u,
+  ERR_RANGE = 8u,
+};
+
+// Per-step quantities live on the device so that a captured step replays
+// correctly.  Written only by single-thread kernels or by one elected thread
+// whose writes no other thread of the same launch reads.
+struct DevState {
+  int step;            // selections completed (t of the step in flight)
+  int n_closed;        // closed blocks per unit
+  int n_last_select;   // n_closed seen by the previous selection
+  int tail_len;        // tokens in the open tail at the start of the step
+  int tail_len_step;   // tail length during the step (tail_len + appended)
+  int gather_count;    // entries in the gather list of the current step
+  unsigned error_bits;
+  int pad;
+};
+
+struct DevStats {
+  unsigned long long steps, selected, hits, misses, fetched_bytes, overlap_sum, overlap_terms;
+  int min_overlap, max_fetch;
+};
+
+// ------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after limit_ns of
+// globaltimer (or a hard iteration cap).  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1; it < (1u << 26); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 127u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+  }
+  return false;
+}
+
+// 2-D tiled TMA load (no multicast) of one box into shared memory, completing
+// on an mbarrier.  x is the innermost coordinate (elements), y the row.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D(16x8, fp32) += A(16x16, bf16, row) * B(16x8, bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 b16 matrix held one row-pair per lane (row lane/4, columns
+// 2*(lane%4) and +1) across the warp.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ double bf16_lo_to_f64(uint32_t w) { return (double)__uint_as_float(w << 16); }
+__device__ __forceinline__ double bf16_hi_to_f64(uint32_t w) {
+  return (double)__uint_as_float(w & 0xFFFF0000u);
+}
+
+// fp64 -> bf16 with round-to-nearest-even, by integer rounding of the fp64
+// significand to the bf16 grid (8 significant bits; spacing 2^-133 below
+// 2^-126), overflow to infinity.
+__device__ __forceinline__ uint32_t f64_to_bf16_bits(double x) {
+  const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
+  const uint32_t sign = static_cast<uint32_t>(u >> 48) & 0x8000u;
+  const unsigned long long mag = u & 0x7FFFFFFFFFFFFFFFull;
+  if (mag > 0x7FF0000000000000ull) return 0x7FC0u;
+  if (mag == 0x7FF0000000000000ull) return sign | 0x7F80u;
+  const int e = static_cast<int>(mag >> 52);
+  if (e == 0) return sign;  // fp64 subnormal: far below half the bf16 spacing
+  const int E = e - 1023;
+  const unsigned long long m = (mag & 0xFFFFFFFFFFFFFull) | (1ull << 52);
+  const int Eq = (E < -126 ? -126 : E) - 7;  // exponent of the bf16 grid spacing
+  const int shift = Eq - (E - 52);           // low significand bits to drop (>= 45)
+  if (shift >= 54) return sign;              // value < half a grid step
+  unsigned long long q = m >> shift;
+  const unsigned long long rem = m & ((1ull << shift) - 1);
+  const unsigned long long half = 1ull << (shift - 1);
+  if (rem > half || (rem == half && (q & 1ull))) ++q;
+  int bits = ((Eq + 7 + 126) << 7) + static_cast<int>(q);
+  if (bits >= 0x7F80) bits = 0x7F80;
+  return sign | static_cast<uint32_t>(bits);
+}
+
+// ------------------------------------------------------------------ launches
+// Each returns the launch error (cudaSuccess if queued).
+
+// Pooled keys of sub-blocks [s_begin, s_end) of every unit.
+// src: bf16 [U, src_unit_tokens, d] (device or mapped host); kbar: bf16
+// [U, kbar_unit_rows, d].
+cudaError_t launch_pool(const uint16_t* src, size_t src_unit_tokens, int U, int s_begin, int s_end,
+                        uint16_t* kbar, int kbar_unit_rows, cudaStream_t st);
+
+struct ScoreArgs {
+  const uint16_t* q;        // [B, Hq, d]
+  const uint16_t* kbar;     // [U, max_blocks*R, d]
+  double* scores;           // [U, max_blocks]
+  const DevState* ds;
+  int U, Hq, Hkv, G, max_blocks;
+};
+cudaError_t launch_score(const ScoreArgs& a, cudaStream_t st);
+
+struct SelectArgs {
+  const float* agnostic;    // [U, max_blocks]
+  const double* scores;     // [U, max_blocks]
+  int* ge;                  // [U, k_e] state, ascending
+  int* prev;                // [U, k] state S(t-1), ascending, -1 pad
+  int* sel;                 // [U, k] output
+  DevState* ds;
+  DevStats* st;
+  int U, max_blocks, k_q, k_e, k, c_max, words;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
+
+struct PlanArgs {
+  const int* sel;           // [U, k]
+  int* fetch;               // [U, k] output, -1 pad
+  int* n_fetch;             // [U] output
+  int* slot_block;          // [U, C]
+  int* last_used;           // [U, C]
+  int* block_slot;          // [U, max_blocks]
+  int* items;               // [U, k] cache slots: hits then misses
+  int* n_hit;               // [U]
+  int* n_items;             // [U]
+  int4* glist;              // [U*k] gather list (unit, block, slot)
+  DevState* ds;
+  DevStats* st;
+  int U, k, C, max_blocks;
+};
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st);
+
+struct GatherArgs {
+  const uint16_t* hk;       // host K (device-addressable), [U, max_blocks*P, d]
+  const uint16_t* hv;
+  uint16_t* ck;             // cache K [U, C, P, d]
+  uint16_t* cv;
+  const int4* glist;
+  const int* count;         // entries to copy (device)
+  DevState* ds;
+  int U, C, max_blocks;
+};
+cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t st);
+
+struct DecodeArgs {
+  const uint16_t* q;        // [B, Hq, d]
+  const int* sel;           // resident: [U, k] block ids
+  const int* items;         // offloaded: [U, k] slots
+  const int* n_hit;         // [U]
+  const int* n_items;       // [U]
+  float* part_o;            // [U, nparts, G, d]
+  float2* part_ml;          // [U, nparts, G]
+  DevState* ds;
+  int U, Hq, Hkv, G, k, max_blocks, C;
+  int resident;             // 1: sel indexes the resident KV
+  int phase;                // 1: hits (+ tail split), 2: misses
+  int splits, bps, part_base, nparts, tail_split;
+};
+struct DecodeMaps {
+  CUtensorMap k, v;         // main K/V: resident KV or the cache, rows of 128 bf16
+  CUtensorMap tk, tv;       // open tail blocks
+};
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st);
+cudaError_t configure_decode();
+
+struct CombineArgs {
+  const float* part_o;
+  const float2* part_ml;
+  uint16_t* out;            // [B, Hq, d]
+  DevState* ds;
+  int U, Hq, Hkv, G, nparts;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+
+struct AppendArgs {
+  const uint16_t* k_new;    // [B, Hkv, d]
+  const uint16_t* v_new;
+  const float* a_close;     // [U] or null
+  uint16_t* tail_k;         // [U, P, d]
+  uint16_t* tail_v;
+  float* a_pending;         // [U]
+  DevState* ds;
+  int U, max_blocks;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
+
+struct CloseArgs {
+  const uint16_t* tail_k;
+  const uint16_t* tail_v;
+  const float* a_pending;
+  uint16_t* kbar;           // [U, max_blocks*R, d]
+  float* agnostic;          // [U, max_blocks]
+  uint16_t* kv_k;           // attached K (host mapped or device) [U, max_blocks*P, d]
+  uint16_t* kv_v;
+  DevState* ds;
+  int U, max_blocks;
+};
+cudaError_t launch_close(const CloseArgs& a, cudaStream_t st);
+
+cudaError_t launch_advance(DevState* ds, DevStats* st, cudaStream_t s);
+cudaError_t launch_init_state(DevState* ds, int n_closed, int tail_len, int step, int n_last_select,
+                              cudaStream_t s);
+cudaError_t launch_reset_stats(DevStats* st, cudaStream_t s);
+cudaError_t launch_wait_flag(const volatile int* flag, DevState* ds, long long timeout_ns, cudaStream_t s);
+
+}  // namespace nosa

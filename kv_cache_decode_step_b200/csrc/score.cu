@@ -1,0 +1,141 @@
+// score.cu -- pooled keys and two-stage block scoring.
+//
+// NOSA: Native and Offloadable Sparse Attention (paperlayer summary), §3.1:
+// blocks are scored in two stages, mean pooling over sub-blocks and then max
+// pooling over the sub-blocks of a block.  Here a sub-block is 16 tokens and a
+// block 64 (4 sub-blocks); the sub-block score of KV head g sums the raw dot
+// products of its G query heads with the pooled key.
+#include "nosa_internal.cuh"
+
+namespace nosa {
+
+// ---------------------------------------------------------------- pooling
+// Block of 256 threads = 16 sub-blocks x 16 lanes; a lane owns 8 dims (16 B).
+// The 16 keys of a sub-block are summed exactly in fp64 (bf16 inputs), divided
+// by 16 (exact) and rounded once to bf16.
+__global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ src, size_t src_unit_tokens,
+                                                   int s_begin, int s_end, uint4* __restrict__ kbar,
+                                                   int kbar_unit_rows) {
+  const int u = blockIdx.y;
+  const int s = s_begin + blockIdx.x * 16 + (threadIdx.x >> 4);
+  if (s >= s_end) return;
+  const int c = threadIdx.x & 15;
+  const uint4* p = src + ((size_t)u * src_unit_tokens + (size_t)s * kQ) * kRowU4 + c;
+  double acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  uint4 w[kQ];
+#pragma unroll
+  for (int j = 0; j < kQ; ++j) w[j] = p[(size_t)j * kRowU4];
+#pragma unroll
+  for (int j = 0; j < kQ; ++j) {
+    acc[0] += bf16_lo_to_f64(w[j].x); acc[1] += bf16_hi_to_f64(w[j].x);
+    acc[2] += bf16_lo_to_f64(w[j].y); acc[3] += bf16_hi_to_f64(w[j].y);
+    acc[4] += bf16_lo_to_f64(w[j].z); acc[5] += bf16_hi_to_f64(w[j].z);
+    acc[6] += bf16_lo_to_f64(w[j].w); acc[7] += bf16_hi_to_f64(w[j].w);
+  }
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = f64_to_bf16_bits(acc[i] * (1.0 / kQ));
+  uint4 r;
+  r.x = o[0] | (o[1] << 16);
+  r.y = o[2] | (o[3] << 16);
+  r.z = o[4] | (o[5] << 16);
+  r.w = o[6] | (o[7] << 16);
+  kbar[((size_t)u * kbar_unit_rows + s) * kRowU4 + c] = r;
+}
+
+cudaError_t launch_pool(const uint16_t* src, size_t src_unit_tokens, int U, int s_begin, int s_end,
+                        uint16_t* kbar, int kbar_unit_rows, cudaStream_t st) {
+  if (s_end <= s_begin || U <= 0) return cudaSuccess;
+  dim3 grid((s_end - s_begin + 15) / 16, U);
+  pool_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(src), src_unit_tokens, s_begin, s_end,
+                                    reinterpret_cast<uint4*>(kbar), kbar_unit_rows);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- scoring
+// One CTA = one unit x 64 blocks; one warp handles one block per iteration:
+// lanes 8r..8r+7 hold sub-block r, lane c-part owns dims [16c, 16c+16).
+// The group's queries are summed first (fp64, exact for bf16 inputs), so each
+// sub-block score is one 128-term fp64 dot product whose products are exact;
+// only the summation order differs from the definition.
+constexpr int kScoreBlocksPerCta = 64;
+
+__device__ __forceinline__ double dot16(const uint4& a, const uint4& b, const double* qt) {
+  double s = 0.0;
+  s = fma(qt[0], bf16_lo_to_f64(a.x), s);  s = fma(qt[1], bf16_hi_to_f64(a.x), s);
+  s = fma(qt[2], bf16_lo_to_f64(a.y), s);  s = fma(qt[3], bf16_hi_to_f64(a.y), s);
+  s = fma(qt[4], bf16_lo_to_f64(a.z), s);  s = fma(qt[5], bf16_hi_to_f64(a.z), s);
+  s = fma(qt[6], bf16_lo_to_f64(a.w), s);  s = fma(qt[7], bf16_hi_to_f64(a.w), s);
+  s = fma(qt[8], bf16_lo_to_f64(b.x), s);  s = fma(qt[9], bf16_hi_to_f64(b.x), s);
+  s = fma(qt[10], bf16_lo_to_f64(b.y), s); s = fma(qt[11], bf16_hi_to_f64(b.y), s);
+  s = fma(qt[12], bf16_lo_to_f64(b.z), s); s = fma(qt[13], bf16_hi_to_f64(b.z), s);
+  s = fma(qt[14], bf16_lo_to_f64(b.w), s); s = fma(qt[15], bf16_hi_to_f64(b.w), s);
+  return s;
+}
+
+__device__ __forceinline__ double block_reduce(double s) {
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 4);
+  double o = __shfl_xor_sync(0xffffffffu, s, 8);
+  s = o > s ? o : s;
+  o = __shfl_xor_sync(0xffffffffu, s, 16);
+  return o > s ? o : s;
+}
+
+__global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
+  const int u = blockIdx.y;
+  const int n = a.ds->n_closed;
+  const int j0 = blockIdx.x * kScoreBlocksPerCta;
+  if (j0 >= n) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = lane >> 3, c = lane & 7;
+  const int b = u / a.Hkv, g = u % a.Hkv;
+
+  double qt[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) qt[i] = 0.0;
+  const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + (size_t)g * a.G) * kD) + 2 * c;
+  for (int h = 0; h < a.G; ++h) {
+    const uint4 x = qrow[h * kRowU4], y = qrow[h * kRowU4 + 1];
+    const uint32_t wv[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      qt[2 * i] += bf16_lo_to_f64(wv[i]);
+      qt[2 * i + 1] += bf16_hi_to_f64(wv[i]);
+    }
+  }
+
+  const uint4* kb = reinterpret_cast<const uint4*>(a.kbar) +
+                    ((size_t)u * a.max_blocks * kR + r) * kRowU4 + 2 * c;
+  double* out = a.scores + (size_t)u * a.max_blocks;
+  const int jend = min(n, j0 + kScoreBlocksPerCta);
+  // two blocks per iteration to keep four 16-byte loads in flight per lane
+  for (int j = j0 + warp; j < jend; j += 16) {
+    const int j2 = j + 8;
+    const uint4* p = kb + (size_t)j * kR * kRowU4;
+    const uint4 a0 = p[0], a1 = p[1];
+    uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+    if (j2 < jend) {
+      const uint4* p2 = kb + (size_t)j2 * kR * kRowU4;
+      b0 = p2[0];
+      b1 = p2[1];
+    }
+    const double s1 = block_reduce(dot16(a0, a1, qt));
+    const double s2 = block_reduce(dot16(b0, b1, qt));
+    if (lane == 0) {
+      out[j] = s1;
+      if (j2 < jend) out[j2] = s2;
+    }
+  }
+}
+
+cudaError_t launch_score(const ScoreArgs& a, cudaStream_t st) {
+  dim3 grid((a.max_blocks + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta, a.U);
+  score_kernel<<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace nosa

@@ -1,0 +1,115 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle
+on the same seeded inputs.  Selections, fetch lists and resident sets must be
+bit-exact; bf16 attention outputs within max-abs 2e-2 and mean-abs 2e-3 of the
+oracle's fp64 result.  The five workloads run at full size (the oracle checks
+a sample of units, every step of their selections)."""
+
+import numpy as np
+import pytest
+
+from kv_cache_decode_step_b200 import configs, inputs
+from gpu_harness import check_all_unit_invariants, compare, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _full(w, sample, attend, graph=False, cache_steps=()):
+    data = inputs.generate(w)
+    rec = run_gpu(w, data, sample, attend, graph=graph, cache_steps=cache_steps)
+    refs = run_oracle(w, data, sample, attend)
+    err = compare(w, rec, refs, sample)
+    check_all_unit_invariants(w, rec, w.steps)
+    print(f"{w.name}: max-abs {err[0]:.3e} mean-abs {err[1]:.3e} stats {rec.stats}")
+    return rec
+
+
+@pytest.mark.parametrize("offloaded", [True, False])
+def test_tiny_all_units_all_steps(offloaded):
+    w = configs.get("tiny")
+    if not offloaded:
+        w = w.with_(offloaded=False, cache_factor=0)
+    _full(w, range(w.units), range(w.steps), cache_steps=range(w.steps))
+
+
+def test_layer8b_resident():
+    w = configs.get("layer8b")
+    _full(w, [0, 37, 64, 127], list(range(0, w.steps, 16)) + [w.steps - 1])
+
+
+def test_offload_b64_graph_replay():
+    w = configs.get("offload_b64")
+    _full(w, [0, 101, 256, 511], list(range(0, w.steps, 32)) + [w.steps - 1], graph=True,
+          cache_steps=[1, 100, w.steps - 1])
+
+
+def test_long_input_offloaded():
+    w = configs.get("long_input")
+    _full(w, [0, 13, 31], list(range(0, w.steps, 16)) + [31, 32, 33, w.steps - 1],
+          cache_steps=[31, 32, w.steps - 1])
+
+
+def test_long_generation_appends_and_closes():
+    w = configs.get("long_gen")
+    attend = [0, 1, 62, 63, 64, 65, 127, 128, 1000, w.steps - 1]
+    rec = _full(w, [0, 77, 255], attend, cache_steps=[64, 1000])
+    assert rec.stats["n_closed"] == w.n_blocks0 + w.steps // w.block
+
+
+# ------------------------------------------------------------------ edge cases
+
+@pytest.mark.parametrize("offloaded", [True, False])
+def test_ragged_prompt_tail(offloaded):
+    """A prompt that ends inside a block: the partial block is attended, never
+    scored or fetched."""
+    w = configs.get("tiny", context=4096 + 37, steps=8)
+    if not offloaded:
+        w = w.with_(offloaded=False, cache_factor=0)
+    _full(w, range(w.units), range(w.steps), cache_steps=[0, 7])
+
+
+def test_ragged_tail_with_appends_closing_a_block():
+    w = configs.get("tiny", context=4096 + 60, steps=12, append=True)
+    rec = _full(w, range(w.units), range(w.steps), cache_steps=[3, 4, 11])
+    assert rec.stats["n_closed"] == 65 and rec.stats["tail_len"] == 8
+
+
+def test_plain_topk_mode_without_agnostic_part():
+    """k_e = 0 and no overlap floor: selection is the plain top-k of scores."""
+    w = configs.get("tiny", k_query=16, k_agnostic=0, min_overlap=0, steps=10)
+    _full(w, range(w.units), range(w.steps))
+
+
+@pytest.mark.parametrize("hq", [2, 4, 16])
+def test_group_sizes(hq):
+    """G = 1, 2 and 8 query heads per KV head."""
+    w = configs.get("tiny", n_q_heads=hq, steps=6)
+    _full(w, range(w.units), range(w.steps))
+
+
+def test_single_split_budget_equals_all_blocks():
+    """Budget covering every block: selection is everything, output is dense."""
+    w = configs.get("tiny", context=16 * 64, k_query=12, k_agnostic=4, steps=5)
+    rec = _full(w, range(w.units), range(w.steps))
+    assert np.array_equal(rec.sel[0, 0], np.arange(16))
+
+
+@pytest.mark.parametrize("offloaded", [True, False])
+def test_maximum_block_count(offloaded):
+    """max_blocks = 8192 (512K tokens per unit), the largest the ABI accepts,
+    with the largest cache (1024 slots)."""
+    w = configs.get("tiny", context=8192 * 64, steps=4, k_query=48, k_agnostic=16, min_overlap=52,
+                    cache_factor=16)
+    if not offloaded:
+        w = w.with_(offloaded=False, cache_factor=0)
+    assert w.max_blocks == 8192
+    _full(w, range(w.units), [0, 3], cache_steps=[3])
+
+
+def test_side_stream_and_single_stream_agree():
+    w = configs.get("tiny", steps=6)
+    data = inputs.generate(w)
+    a = run_gpu(w, data, range(w.units), range(w.steps), side_copy_stream=True)
+    b = run_gpu(w, data, range(w.units), range(w.steps), side_copy_stream=False)
+    assert np.array_equal(a.sel, b.sel) and np.array_equal(a.fetch, b.fetch)
+    for t in a.out:
+        assert np.array_equal(a.out[t], b.out[t])
