@@ -42,7 +42,7 @@ HBM_NOMINAL_GBS = 8000.0
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--steps", type=int, default=4000)
     p.add_argument("--warmup", type=int, default=8)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="offload_b64")
@@ -60,9 +60,10 @@ def dist_env():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms; only the
+    samples whose timestamps fall inside the timed window are summarised."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -70,6 +71,7 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
@@ -77,40 +79,70 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.STDOUT)
         except Exception:
             self.proc = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
             return None
+        time.sleep(0.25)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.f.close()
-        sm, smax, reasons = [], [], set()
+        import datetime
+        sm, smax, pw, reasons, n_all = [], [], [], set(), 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, cmax = float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            n_all += 1
+            if self.t0 is not None and not (self.t0 <= ts <= self.t1):
+                continue
+            sm.append(clk)
+            smax.append(cmax)
+            try:
+                pw.append(float(parts[4]))
+            except ValueError:
+                pass
+            for n, v in zip(names, parts[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
-            return None
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "samples_total": n_all}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w_max": max(pw) if pw else None}
 
 
 # ------------------------------------------------------------------ helpers
+def max_over_ranks(torch, dist, ms_local, device, world):
+    """The slowest rank's timed-region length (every rank takes part)."""
+    t = torch.tensor([float(ms_local)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, batch, steps, ms_max):
+    """Whole-job throughput: every rank decodes `batch` tokens per step."""
+    return world * batch * steps / (ms_max * 1e-3)
+
+
 def measured_peaks():
     try:
         return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -166,10 +198,10 @@ def cpu_baseline(w, target_s=12.0):
         _, _, _, th = oracle.run_units(cfg, d["k"], d["v"], d["a"], d["q"], attend_steps=None)
         return time.perf_counter() - t0, th
 
-    t_probe, th = run(min(w.units, 16), 2)
-    per_unit_step = t_probe / (min(w.units, 16) * 2)
-    n_units = min(w.units, 64)
-    steps = max(2, min(64, int(target_s / max(per_unit_step * n_units, 1e-6))))
+    t_probe, th = run(min(w.units, 32), 4)
+    per_unit_step = t_probe / (min(w.units, 32) * 4)  # wall time per unit-step, all cores
+    n_units = w.units
+    steps = max(2, min(256, int(target_s / max(per_unit_step * n_units, 1e-6))))
     t, th = run(n_units, steps)
     step_time = t / steps * (w.units / n_units)
     return (w.batch / step_time, th,
@@ -229,7 +261,7 @@ def run_ours(args):
     build.build()
 
     base = configs.get(args.workload)
-    total = 1 + args.warmup + args.steps + args.e2e_steps + 64
+    total = 1 + args.warmup + 1 + args.steps + 2 * min(args.steps, 50) + args.e2e_steps + 8
     w = base.with_(steps=max(base.steps, total))
     data = inputs.generate(w)
     dec = runner.Decoder(w, data, device=local)
@@ -248,27 +280,27 @@ def run_ours(args):
     # ---- timed region: K graph replays
     clocks = ClockSampler(local)
     clocks.start()
+    time.sleep(1.0)  # let the sampler start before the timed window
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    clocks.mark_start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(dec.stream)
     for _ in range(args.steps):
         dec.replay()
     e1.record(dec.stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     st = dec.stats()
     dec.check()
-    t_max = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    ms_max = float(t_max.item())
+    ms_max = max_over_ranks(torch, dist, ms, dev, world)
     ms_step = ms_max / args.steps
-    value = world * w.batch * args.steps / (ms_max * 1e-3)
+    value = job_tokens_per_s(world, w.batch, args.steps, ms_max)
 
     fetched_blocks = st["misses"] / args.steps
     pcie_bytes = st["fetched_bytes"] / args.steps
@@ -281,15 +313,20 @@ def run_ours(args):
     t_pcie = pcie_bytes / (h2d_peak * 1e9)
     step_s = ms_step * 1e-3
 
-    # ---- instrumented pass: same graph, per-phase events per step
-    phase = instrumented_pass(torch, dec, w, nosa, n=min(args.steps, 50))
+    # ---- instrumented passes: per-phase events between the ABI calls.  With
+    # the side copy stream the gather's own duration is visible; with a single
+    # stream the attention launches no longer wait on it.
+    phase = instrumented_pass(torch, dec, w, nosa, n=min(args.steps, 50), single_stream=False)
+    phase1 = instrumented_pass(torch, dec, w, nosa, n=min(args.steps, 50), single_stream=True)
+    phase["attention_ms"] = phase1["decode_ms"]
+    phase["single_stream_step_ms"] = phase1["step_ms"]
 
     # ---- end to end through host buffers: q from pinned host, out to pinned host
     e2e = e2e_pass(torch, dec, w, nosa, args.e2e_steps)
 
     launches_per_step = 8  # score, select, plan, gather, attend x2, combine, advance
     gather_ms = phase["gather_ms"]
-    attn_ms = phase["decode_ms"]
+    attn_ms = phase["attention_ms"]
     gather_gbs = (phase["fetched_bytes_per_step"] / (gather_ms * 1e-3) / 1e9) if gather_ms > 0 else 0.0
     attn_bytes = w.units * w.k * w.block * w.head_dim * 2 * 2 + w.batch * w.n_q_heads * w.head_dim * 2 * 2
     attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9 if attn_ms > 0 else 0.0
@@ -297,7 +334,7 @@ def run_ours(args):
                  "unit": "GB/s", "frac": gather_gbs / h2d_peak if h2d_peak else None, "traffic": None,
                  "peak_source": "pinned cudaMemcpyAsync H2D measured in this run (256 MiB)",
                  "bytes_per_launch": phase["fetched_bytes_per_step"], "ms_per_launch": gather_ms}
-    rl_attn = {"kernel": "decode_kernel+combine_kernel", "bound": "hbm", "achieved": attn_gbs,
+    rl_attn = {"kernel": "decode_kernel x2 + combine_kernel + advance_kernel", "bound": "hbm", "achieved": attn_gbs,
                "peak": hbm_meas, "unit": "GB/s", "frac": attn_gbs / hbm_meas, "traffic": None,
                "peak_source": f"hbm_gbs {hbm_src}", "bytes_per_launch": attn_bytes, "ms_per_launch": attn_ms}
     dominant, other = (rl_gather, rl_attn) if gather_ms >= attn_ms else (rl_attn, rl_gather)
@@ -350,10 +387,11 @@ def run_ours(args):
     return result
 
 
-def instrumented_pass(torch, dec, w, nosa, n):
-    """Replay the same step n times with events between the ABI calls (eager
-    issue on the same streams) and read per-phase durations after each step."""
-    s, cs = dec.stream, dec.copy_stream
+def instrumented_pass(torch, dec, w, nosa, n, single_stream):
+    """Run n more steps eagerly with events between the ABI calls and read the
+    per-phase durations after each step."""
+    s = dec.stream
+    cs = s if single_stream else dec.copy_stream
     ev = {k: torch.cuda.Event(enable_timing=True) for k in ("a", "b", "c", "d", "g", "e")}
     acc = {"score_ms": 0.0, "select_ms": 0.0, "plan_ms": 0.0, "gather_ms": 0.0, "decode_ms": 0.0, "step_ms": 0.0}
     misses0 = dec.stats()["fetched_bytes"]
@@ -382,8 +420,8 @@ def instrumented_pass(torch, dec, w, nosa, n):
     out = {k: v / n for k, v in acc.items()}
     out["fetched_bytes_per_step"] = (dec.stats()["fetched_bytes"] - misses0) / n
     out["steps"] = n
-    out["note"] = ("decode_ms spans attention over hits (overlapping the gather), the wait for the "
-                   "gather, attention over misses, combine and step advance")
+    out["note"] = ("decode_ms spans both attention launches, combine and step advance (with a side copy "
+                   "stream it also holds the wait for the gather)")
     return out
 
 

@@ -29,6 +29,7 @@ from typing import Dict, Iterable, Optional, Sequence
 
 import numpy as np
 import torch
+from scipy.signal import lfilter
 
 from .configs import Workload
 
@@ -73,21 +74,70 @@ def unit_agnostic(w: Workload, u: int) -> np.ndarray:
     return _rng(w, STREAM_AGNOSTIC, u).random(w.max_blocks, dtype=np.float32)
 
 
-def unit_queries(w: Workload, u: int) -> np.ndarray:
-    """bf16 bits [steps, group, head_dim]: the query heads of unit u, per step."""
+def _query_draws(w: Workload, u: int):
+    """q_0 and the innovations eps_1 .. eps_{steps-1} of unit u (fp64), in the
+    order the stream yields them."""
     r = _rng(w, STREAM_QUERY, u)
     shape = (w.group, w.head_dim)
-    q = r.standard_normal(shape)  # fp64
-    out = np.empty((w.steps,) + shape, dtype=np.float64)
-    for t in range(w.steps):
-        if t > 0:
-            eps = r.standard_normal(shape)
-            if w.resample_every and t % w.resample_every == 0:
-                q = eps
-            else:
-                q = w.rho * q + w.sigma * eps
-        out[t] = q
-    return f32_to_bf16_bits(out.astype(np.float32))
+    q0 = r.standard_normal(shape)
+    eps = r.standard_normal((max(w.steps - 1, 0),) + shape)
+    return q0, eps
+
+
+def _queries_from_draws(w: Workload, q0: np.ndarray, eps: np.ndarray) -> np.ndarray:
+    """AR(1) recurrence over a leading batch of units: q0 [n, G, d], eps
+    [n, steps-1, G, d] -> fp64 [n, steps, G, d].
+
+    q_t = rho*q_{t-1} + sigma*eps_t, restarted at q_t = eps_t on resample steps.
+    Each segment between restarts is one linear filter along time (the same two
+    fp64 products and one sum per step as the plain loop)."""
+    n = q0.shape[0]
+    S = w.steps
+    out = np.empty((n, S) + q0.shape[1:], dtype=np.float64)
+    if S == 0:
+        return out
+    out[:, 0] = q0
+    starts = [1] + ([t for t in range(1, S) if w.resample_every and t % w.resample_every == 0])
+    starts = sorted(set(starts))
+    bounds = starts + [S]
+    prev = q0
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        if a >= b:
+            continue
+        x = eps[:, a - 1:b - 1]
+        if w.resample_every and a % w.resample_every == 0:
+            out[:, a] = x[:, 0]
+            if b > a + 1:
+                zi = (w.rho * x[:, 0])[:, None]
+                out[:, a + 1:b] = lfilter([w.sigma], [1.0, -w.rho], x[:, 1:], axis=1, zi=zi)[0]
+        else:
+            zi = (w.rho * prev)[:, None]
+            out[:, a:b] = lfilter([w.sigma], [1.0, -w.rho], x, axis=1, zi=zi)[0]
+        prev = out[:, b - 1]
+    return out
+
+
+def _queries_loop(w: Workload, q0: np.ndarray, eps: np.ndarray) -> np.ndarray:
+    """The same recurrence as a plain per-step loop (kept for cross-checks)."""
+    out = np.empty((q0.shape[0], w.steps) + q0.shape[1:], dtype=np.float64)
+    q = q0
+    if w.steps > 0:
+        out[:, 0] = q
+    for t in range(1, w.steps):
+        e = eps[:, t - 1]
+        q = e if (w.resample_every and t % w.resample_every == 0) else w.rho * q + w.sigma * e
+        out[:, t] = q
+    return out
+
+
+def unit_queries(w: Workload, u: int) -> np.ndarray:
+    """bf16 bits [steps, group, head_dim]: the query heads of unit u, per step."""
+    q0, eps = _query_draws(w, u)
+    q = _queries_from_draws(w, q0[None], eps[None])[0]
+    return f32_to_bf16_bits(q.astype(np.float32))
+
+
+_QCHUNK = 16
 
 
 def _threads() -> int:
@@ -122,15 +172,23 @@ def generate(w: Workload, units: Optional[Sequence[int]] = None,
             out["v"][i] = unit_kv(w, u, "v")
         if "a" in parts:
             out["a"][i] = unit_agnostic(w, u)
-        if "q" in parts:
-            out["q"][i] = unit_queries(w, u)
 
-    if nu <= 2:
-        for i in range(nu):
-            one(i)
+    def queries(i0: int) -> None:
+        # the recurrence runs vectorised over a chunk of units
+        chunk = list(range(i0, min(nu, i0 + _QCHUNK)))
+        draws = [_query_draws(w, units[i]) for i in chunk]
+        q = _queries_from_draws(w, np.stack([d[0] for d in draws]), np.stack([d[1] for d in draws]))
+        out["q"][chunk[0]:chunk[-1] + 1] = f32_to_bf16_bits(q.astype(np.float32))
+
+    jobs = [(one, i) for i in range(nu)]
+    if "q" in parts:
+        jobs += [(queries, i0) for i0 in range(0, nu, _QCHUNK)]
+    if len(jobs) <= 2:
+        for f, i in jobs:
+            f(i)
     else:
         with cf.ThreadPoolExecutor(_threads()) as ex:
-            list(ex.map(one, range(nu)))
+            list(ex.map(lambda j: j[0](j[1]), jobs))
     return out
 
 
