@@ -33,7 +33,7 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_take_the_slowest_time():
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
