@@ -243,8 +243,8 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   c->gather_grid = sms;
   if (const char* v = getenv("NOSA_GATHER_CTAS")) c->gather_grid = atoi(v) > 0 ? atoi(v) : sms;
   c->S1 = (c->k + c->bps - 1) / c->bps;
-  c->S2 = c->offloaded ? c->S1 : 0;
-  c->nparts = c->S1 + 1 + c->S2;
+  c->S2 = c->offloaded ? 1 : 0;
+  c->nparts = c->S1 + 1;
 
   const size_t U = c->U, MB = c->max_blocks, K = c->k;
 #define ALLOC(ptr, n)                    \
@@ -548,24 +548,29 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
   a.tail_split = 1;
   NOSA_CUDA(launch_decode(a, c->maps, st));
   if (c->offloaded) {
+    // phase 2: one CTA per unit attends to its fetched blocks once the gather
+    // has landed and merges every partial of the unit into the output
     if (c->gather_on_side) NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
     a.phase = 2;
-    a.splits = c->S2;
+    a.splits = 1;
     a.part_base = c->S1 + 1;
     a.tail_split = 0;
+    a.merge_out = 1;
+    a.out = static_cast<uint16_t*>(out);
     NOSA_CUDA(launch_decode(a, c->maps, st));
+  } else {
+    CombineArgs cb{};
+    cb.part_o = c->part_o;
+    cb.part_ml = c->part_ml;
+    cb.out = static_cast<uint16_t*>(out);
+    cb.ds = c->ds;
+    cb.U = c->U;
+    cb.Hq = c->cfg.n_q_heads;
+    cb.Hkv = c->cfg.n_kv_heads;
+    cb.G = c->G;
+    cb.nparts = c->nparts;
+    NOSA_CUDA(launch_combine(cb, st));
   }
-  CombineArgs cb{};
-  cb.part_o = c->part_o;
-  cb.part_ml = c->part_ml;
-  cb.out = static_cast<uint16_t*>(out);
-  cb.ds = c->ds;
-  cb.U = c->U;
-  cb.Hq = c->cfg.n_q_heads;
-  cb.Hkv = c->cfg.n_kv_heads;
-  cb.G = c->G;
-  cb.nparts = c->nparts;
-  NOSA_CUDA(launch_combine(cb, st));
   if (c->appends_enabled) {
     CloseArgs cl{};
     cl.tail_k = c->tail_k;

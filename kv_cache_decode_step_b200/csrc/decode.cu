@@ -38,6 +38,45 @@ struct DecSmemLayout {
 
 int decode_smem_bytes() { return DecSmemLayout::kBytes + 1024; }
 
+// Final merge of one unit: the partials of parts [0, part_base) already in
+// global memory plus (optionally) this CTA's four warps' states in shared
+// memory; writes out[b, g*G + h, :] as bf16.
+__device__ void merge_and_store(const DecodeArgs& a, int u, int b, int g, const float* sO, const float* sM,
+                                const float* sL) {
+  const float* po = a.part_o + (size_t)u * a.nparts * a.G * kD;
+  const float2* pml = a.part_ml + (size_t)u * a.nparts * a.G;
+  for (int idx = threadIdx.x; idx < a.G * kD; idx += blockDim.x) {
+    const int h = idx / kD, dd = idx % kD;
+    float M = -INFINITY;
+    for (int p = 0; p < a.part_base; ++p) M = fmaxf(M, pml[p * a.G + h].x);
+    if (sM) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, sM[w * kMaxG + h]);
+    }
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float num = 0.f, den = 0.f;
+    for (int p = 0; p < a.part_base; ++p) {
+      const float2 ml = pml[p * a.G + h];
+      if (ml.y <= 0.f) continue;
+      const float f = exp2f(ml.x - Mu);
+      num += f * po[((size_t)p * a.G + h) * kD + dd];
+      den += f * ml.y;
+    }
+    if (sM) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float l = sL[w * kMaxG + h];
+        if (l <= 0.f) continue;
+        const float f = exp2f(sM[w * kMaxG + h] - Mu);
+        num += f * sO[(w * kMaxG + h) * kD + dd];
+        den += f * l;
+      }
+    }
+    const float r = den > 0.f ? num / den : 0.f;
+    a.out[((size_t)b * a.Hq + (size_t)g * a.G + h) * kD + dd] = (uint16_t)(pack_bf16x2(r, 0.f) & 0xFFFFu);
+  }
+}
+
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                   const __grid_constant__ CUtensorMap map_tk, const __grid_constant__ CUtensorMap map_tv,
@@ -64,22 +103,31 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       base_lo = a.n_hit[u];
       base_hi = a.n_items[u];
     }
-    lo = base_lo + s * a.bps;
-    hi = min(base_lo + (s + 1) * a.bps, base_hi);
+    if (a.merge_out) {  // one CTA per unit takes every remaining item
+      lo = base_lo;
+      hi = base_hi;
+    } else {
+      lo = base_lo + s * a.bps;
+      hi = min(base_lo + (s + 1) * a.bps, base_hi);
+    }
   }
   const int n_it = hi > lo ? hi - lo : 0;
   const size_t part = (size_t)u * a.nparts + a.part_base + s;
   float* po = a.part_o + part * a.G * kD;
   float2* pml = a.part_ml + part * a.G;
-  if (n_it == 0) {
-    if (threadIdx.x < a.G) pml[threadIdx.x] = make_float2(-INFINITY, 0.f);
-    return;
-  }
 
   extern __shared__ unsigned char dsm_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
                                                        ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + DecSmemLayout::kBars);
+  if (n_it == 0) {
+    if (a.merge_out) {
+      merge_and_store(a, u, b, g, nullptr, nullptr, nullptr);
+    } else if (threadIdx.x < a.G) {
+      pml[threadIdx.x] = make_float2(-INFINITY, 0.f);
+    }
+    return;
+  }
 
   // ---- producer: thread 0 issues one block's K and V (4 boxes, 32 KiB)
   auto issue = [&](int it, int st) {
@@ -217,7 +265,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         (void)mbar_wait_bounded(&bars[it % kStages], (uint32_t)((it / kStages) & 1), kWaitLimitNs);
     }
     __syncthreads();
-    if (threadIdx.x < a.G) pml[threadIdx.x] = make_float2(-INFINITY, 0.f);
+    if (!a.merge_out && threadIdx.x < a.G) pml[threadIdx.x] = make_float2(-INFINITY, 0.f);
     return;
   }
 
@@ -245,6 +293,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     w[h1 * kD + d0 + 8] = o[mt][3];
   }
   __syncthreads();
+  if (a.merge_out) {
+    merge_and_store(a, u, b, g, sO, sM, sL);
+    return;
+  }
   for (int idx = threadIdx.x; idx < a.G * kD; idx += kDecThreads) {
     const int h = idx / kD, dd = idx % kD;
     float M = -INFINITY;

@@ -18,13 +18,17 @@ namespace nosa {
 constexpr int kPlanWarps = 4;
 constexpr unsigned kAll = 0xffffffffu;
 
+// One warp per unit.  The unit's slot tables are staged in shared memory so
+// the only dependent global round trips are sel -> block_slot.
 __global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(PlanArgs a) {
   extern __shared__ int sm_plan[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * kPlanWarps + warp;
   if (u >= a.U) return;
-  int* smiss = sm_plan + (size_t)warp * 2 * a.k;  // missed blocks, ascending
-  int* ssrc = smiss + a.k;                         // slots they will take
+  int* sb = sm_plan + (size_t)warp * (2 * a.C + 2 * a.k);  // slot -> block
+  int* lu = sb + a.C;                                       // slot -> last step selected
+  int* smiss = lu + a.C;                                    // missed blocks, ascending
+  int* ssrc = smiss + a.k;                                  // slots they will take
 
   const int t = a.ds->step;
   const int* sel = a.sel + (size_t)u * a.k;
@@ -34,6 +38,12 @@ __global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(PlanArgs a) {
   int* items = a.items + (size_t)u * a.k;
   const unsigned lt = (1u << lane) - 1u;
 
+  for (int c = lane; c < a.C; c += 32) {
+    sb[c] = slot_block[c];
+    lu[c] = last_used[c];
+  }
+  __syncwarp();
+
   // 1. hits refresh their stamp; misses are listed in ascending order
   int n_hit = 0, n_miss = 0;
   for (int i0 = 0; i0 < a.k; i0 += 32) {
@@ -41,10 +51,11 @@ __global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(PlanArgs a) {
     const int bj = i < a.k ? sel[i] : -1;
     const bool valid = bj >= 0 && bj < a.max_blocks;
     const int slot = valid ? block_slot[bj] : -1;
-    const bool hit = valid && slot >= 0;
-    const bool miss = valid && slot < 0;
+    const bool hit = valid && slot >= 0 && slot < a.C;
+    const bool miss = valid && !hit;
     const unsigned hm = __ballot_sync(kAll, hit), mm = __ballot_sync(kAll, miss);
     if (hit) {
+      lu[slot] = t;
       last_used[slot] = t;
       items[n_hit + __popc(hm & lt)] = slot;
     }
@@ -58,7 +69,7 @@ __global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(PlanArgs a) {
   int n_src = 0;
   for (int c0 = 0; c0 < a.C && n_src < n_miss; c0 += 32) {
     const int c = c0 + lane;
-    const bool fr = c < a.C && slot_block[c] < 0;
+    const bool fr = c < a.C && sb[c] < 0;
     const unsigned fm = __ballot_sync(kAll, fr);
     const int pos = n_src + __popc(fm & lt);
     if (fr && pos < n_miss) ssrc[pos] = c;
@@ -67,35 +78,35 @@ __global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(PlanArgs a) {
   n_src = min(n_src, n_miss);
   __syncwarp();
 
-  // 3. victims: resident, not selected now (stamp < t), oldest stamp first
+  // 3. victims: resident, not selected now (stamp < t); least recent stamp,
+  //    then lower block id, first.  Stamps are >= 0 for resident slots.
   bool failed = false;
   while (n_src < n_miss) {
-    unsigned long long best = ~0ull;
+    unsigned bhi = 0xffffffffu, blo = 0xffffffffu;
     for (int c = lane; c < a.C; c += 32) {
-      const int bj = slot_block[c];
-      const int lu = last_used[c];
-      if (bj >= 0 && lu < t) {
-        const unsigned long long key =
-            ((unsigned long long)(unsigned)lu << 32) | (unsigned long long)(unsigned)bj;
-        if (key < best) best = key;
+      const int bj = sb[c];
+      const int st = lu[c];
+      if (bj >= 0 && st < t) {
+        const unsigned h = (unsigned)st, l = (unsigned)bj;
+        if (h < bhi || (h == bhi && l < blo)) {
+          bhi = h;
+          blo = l;
+        }
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long ob = __shfl_xor_sync(kAll, best, o);
-      best = ob < best ? ob : best;
-    }
-    if (best == ~0ull) {
+    const unsigned mhi = __reduce_min_sync(kAll, bhi);
+    const unsigned mlo = __reduce_min_sync(kAll, bhi == mhi ? blo : 0xffffffffu);
+    if (mhi == 0xffffffffu) {
       failed = true;
       break;
     }
     if (lane == 0) {
-      const int victim_block = (int)(unsigned)(best & 0xffffffffull);
+      const int victim_block = (int)mlo;
       const int vslot = block_slot[victim_block];
       ssrc[n_src] = vslot;
       block_slot[victim_block] = -1;
-      slot_block[vslot] = -2;  // claimed; excluded from the search
-      last_used[vslot] = t;
+      sb[vslot] = -2;  // claimed; excluded from the search
+      lu[vslot] = t;
     }
     ++n_src;
     __syncwarp();
@@ -136,7 +147,11 @@ __global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(PlanArgs a) {
 
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st) {
   const int grid = (a.U + kPlanWarps - 1) / kPlanWarps;
-  const size_t smem = (size_t)kPlanWarps * 2 * a.k * sizeof(int);
+  const size_t smem = (size_t)kPlanWarps * (2 * a.C + 2 * a.k) * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
   plan_kernel<<<grid, kPlanWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
@@ -185,9 +200,25 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
   }
 }
 
+// The gather is launched with the device's highest CTA priority so that its
+// few CTAs are dispatched ahead of the attention CTAs that run concurrently
+// on the compute stream; otherwise the PCIe transfer starts only once
+// attention has drained.
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t st) {
-  gather_kernel<<<grid, kGatherThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  int least = 0, greatest = 0;
+  cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGatherThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributePriority;
+  attr[0].val.priority = greatest;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gather_kernel, a);
 }
 
 }  // namespace nosa

@@ -242,6 +242,8 @@ struct DecodeArgs {
   int resident;             // 1: sel indexes the resident KV
   int phase;                // 1: hits (+ tail split), 2: misses
   int splits, bps, part_base, nparts, tail_split;
+  int merge_out;            // 1: one CTA per unit, merge parts [0, part_base) and write out
+  uint16_t* out;            // [B, Hq, d] when merge_out
 };
 struct DecodeMaps {
   CUtensorMap k, v;         // main K/V: resident KV or the cache, rows of 128 bf16

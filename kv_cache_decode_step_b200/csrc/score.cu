@@ -55,8 +55,8 @@ cudaError_t launch_pool(const uint16_t* src, size_t src_unit_tokens, int U, int 
 }
 
 // ---------------------------------------------------------------- scoring
-// One CTA = one unit x 64 blocks; one warp handles one block per iteration:
-// lanes 8r..8r+7 hold sub-block r, lane c-part owns dims [16c, 16c+16).
+// One CTA = one unit x 64 blocks.  Within a block, lanes 8r..8r+7 hold
+// sub-block r and lane 8r+c owns dims [16c, 16c+16).
 // The group's queries are summed first (fp64, exact for bf16 inputs), so each
 // sub-block score is one 128-term fp64 dot product whose products are exact;
 // only the summation order differs from the definition.
@@ -85,22 +85,39 @@ __device__ __forceinline__ double block_reduce(double s) {
   return o > s ? o : s;
 }
 
+// Each warp owns 8 consecutive blocks (8 KiB of pooled keys) and issues all of
+// their loads before any arithmetic, so every SM keeps tens of KiB in flight.
+constexpr int kScoreBlocksPerWarp = kScoreBlocksPerCta / 8;
+
 __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
   const int u = blockIdx.y;
   const int n = a.ds->n_closed;
-  const int j0 = blockIdx.x * kScoreBlocksPerCta;
-  if (j0 >= n) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = blockIdx.x * kScoreBlocksPerCta + warp * kScoreBlocksPerWarp;
+  if (j0 >= n) return;
   const int r = lane >> 3, c = lane & 7;
   const int b = u / a.Hkv, g = u % a.Hkv;
+
+  const uint4* kb = reinterpret_cast<const uint4*>(a.kbar) +
+                    ((size_t)u * a.max_blocks * kR + (size_t)j0 * kR + r) * kRowU4 + 2 * c;
+  uint4 x[kScoreBlocksPerWarp][2];
+#pragma unroll
+  for (int i = 0; i < kScoreBlocksPerWarp; ++i) {
+    if (j0 + i < n) {
+      x[i][0] = kb[(size_t)i * kR * kRowU4];
+      x[i][1] = kb[(size_t)i * kR * kRowU4 + 1];
+    } else {
+      x[i][0] = x[i][1] = make_uint4(0, 0, 0, 0);
+    }
+  }
 
   double qt[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) qt[i] = 0.0;
   const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + (size_t)g * a.G) * kD) + 2 * c;
   for (int h = 0; h < a.G; ++h) {
-    const uint4 x = qrow[h * kRowU4], y = qrow[h * kRowU4 + 1];
-    const uint32_t wv[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+    const uint4 y0 = qrow[h * kRowU4], y1 = qrow[h * kRowU4 + 1];
+    const uint32_t wv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       qt[2 * i] += bf16_lo_to_f64(wv[i]);
@@ -108,27 +125,18 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
     }
   }
 
-  const uint4* kb = reinterpret_cast<const uint4*>(a.kbar) +
-                    ((size_t)u * a.max_blocks * kR + r) * kRowU4 + 2 * c;
-  double* out = a.scores + (size_t)u * a.max_blocks;
-  const int jend = min(n, j0 + kScoreBlocksPerCta);
-  // two blocks per iteration to keep four 16-byte loads in flight per lane
-  for (int j = j0 + warp; j < jend; j += 16) {
-    const int j2 = j + 8;
-    const uint4* p = kb + (size_t)j * kR * kRowU4;
-    const uint4 a0 = p[0], a1 = p[1];
-    uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
-    if (j2 < jend) {
-      const uint4* p2 = kb + (size_t)j2 * kR * kRowU4;
-      b0 = p2[0];
-      b1 = p2[1];
-    }
-    const double s1 = block_reduce(dot16(a0, a1, qt));
-    const double s2 = block_reduce(dot16(b0, b1, qt));
-    if (lane == 0) {
-      out[j] = s1;
-      if (j2 < jend) out[j2] = s2;
-    }
+  double sres[kScoreBlocksPerWarp];
+#pragma unroll
+  for (int i = 0; i < kScoreBlocksPerWarp; ++i) sres[i] = dot16(x[i][0], x[i][1], qt);
+#pragma unroll
+  for (int i = 0; i < kScoreBlocksPerWarp; ++i) sres[i] = block_reduce(sres[i]);
+  if (lane < kScoreBlocksPerWarp) {
+    // lane i writes block j0 + i (all lanes hold every reduced value)
+    double v = sres[0];
+#pragma unroll
+    for (int i = 1; i < kScoreBlocksPerWarp; ++i)
+      if (lane == i) v = sres[i];
+    if (j0 + lane < n) a.scores[(size_t)u * a.max_blocks + j0 + lane] = v;
   }
 }
 

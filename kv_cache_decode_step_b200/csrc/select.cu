@@ -14,10 +14,13 @@
 //   c_t        = max(0, (k - m) - |Gamma_e(t) \ S(t-1)|), unbounded at t = 0
 //   Gamma_q(t) = top-k_q by score of (S(t-1) \ Gamma_e(t)) ∪ top-c_t(new)
 //   S(t)       = Gamma_e(t) ∪ Gamma_q(t), ties to the lower block id.
-// Sets are bitmaps in shared memory; lane l owns blocks j with j % 32 == l, so
-// bit l of word i is block 32 i + l.  A top-c pass keeps each lane's best
-// remaining candidate and, per round, reduces the warp's best with shuffles;
-// only the winner's lane rescans its blocks.
+//
+// Sets are bitmaps in shared memory; lane l owns the blocks j with j % 32 == l
+// (bit l of word j / 32).  Keys are order-preserving integer images of the
+// scores (larger score -> larger key), so one warp-wide argmax is two
+// redux.sync max steps, a ballot and, only on an exact tie, a redux.sync min
+// over block ids.  Choosing c of a set of p candidates takes min(c, p - c)
+// rounds: either move the c best out, or remove the p - c worst.
 #include <climits>
 
 #include "nosa_internal.cuh"
@@ -26,6 +29,7 @@ namespace nosa {
 
 constexpr int kSelWarps = 4;
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kSmemKeys = 1024;  // query-aware keys staged in shared memory up to this many blocks
 
 __device__ __forceinline__ unsigned valid_bits(int w, int n) {
   const int lo = w * 32;
@@ -34,55 +38,105 @@ __device__ __forceinline__ unsigned valid_bits(int w, int n) {
   return (1u << (n - lo)) - 1u;
 }
 
-// Better = larger key, then smaller id.
-__device__ __forceinline__ bool better(double v, int i, double bv, int bi) {
-  return v > bv || (v == bv && i < bi);
+// Order-preserving maps to unsigned integers.  No real key maps to 0, which
+// marks "no candidate".
+__device__ __forceinline__ unsigned long long key_f64(double x) {
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
+  return (b & 0x8000000000000000ull) ? ~b : (b | 0x8000000000000000ull);
+}
+__device__ __forceinline__ unsigned long long key_f32(float x) {
+  const unsigned b = __float_as_uint(x);
+  return (unsigned long long)((b & 0x80000000u) ? ~b : (b | 0x80000000u)) << 32;
 }
 
-template <typename KeyF>
-__device__ __forceinline__ void lane_best(const unsigned* mask, int words, int lane, KeyF key, double& bv,
-                                          int& bi) {
-  bv = -INFINITY;
-  bi = INT_MAX;
+// Key source for a selection: staged 64-bit keys in shared memory, or the
+// fp32 agnostic scores / fp64 scores in global memory.  `worst` flips the
+// order (smallest score first, ties to the larger block id).
+struct Keys {
+  const unsigned long long* smem;
+  const float* ag;
+  const double* sc;
+  bool worst;
+  __device__ __forceinline__ unsigned long long raw(int j) const {
+    if (smem) return smem[j];
+    if (ag) return key_f32(ag[j]);
+    return key_f64(sc[j]);
+  }
+  __device__ __forceinline__ unsigned long long operator()(int j) const {
+    const unsigned long long k = raw(j);
+    return worst ? ~k : k;
+  }
+  // tie order: smaller tie wins
+  __device__ __forceinline__ unsigned tie(int j) const { return worst ? ~(unsigned)j : (unsigned)j; }
+};
+
+// This lane's best remaining candidate of `mask`.  Key 0 = none.
+__device__ __forceinline__ void lane_best(const unsigned* mask, int words, int lane, const Keys& K,
+                                          unsigned long long& bk, int& bj) {
+  bk = 0ull;
+  bj = -1;
   for (int w = 0; w < words; ++w) {
     if ((mask[w] >> lane) & 1u) {
       const int j = w * 32 + lane;
-      const double v = key(j);
-      if (bi == INT_MAX || v > bv) {  // ascending j: equal keys keep the first
-        bv = v;
-        bi = j;
+      const unsigned long long k = K(j);
+      if (bj < 0 || k > bk || (k == bk && K.tie(j) < K.tie(bj))) {
+        bk = k;
+        bj = j;
       }
     }
   }
 }
 
-// Move the `cnt` best blocks of `mask` into `out` (both bitmaps).
-template <typename KeyF>
-__device__ void warp_topk(unsigned* mask, unsigned* out, int words, int cnt, int lane, KeyF key) {
-  if (cnt <= 0) return;
-  double bv;
-  int bi;
-  lane_best(mask, words, lane, key, bv, bi);
-  for (int r = 0; r < cnt; ++r) {
-    double v = bv;
-    int i = bi;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ov = __shfl_xor_sync(kFull, v, o);
-      const int oi = __shfl_xor_sync(kFull, i, o);
-      if (oi != INT_MAX && (i == INT_MAX || better(ov, oi, v, i))) {
-        v = ov;
-        i = oi;
-      }
-    }
-    if (i == INT_MAX) break;  // no candidates left (same on every lane)
-    if ((i & 31) == lane) {
-      mask[i >> 5] &= ~(1u << lane);
-      out[i >> 5] |= (1u << lane);
-      lane_best(mask, words, lane, key, bv, bi);
+// Warp-wide winner of (key max, tie min); -1 when every lane is empty.
+__device__ __forceinline__ int warp_winner(unsigned long long bk, int bj, const Keys& K, int lane) {
+  const unsigned hi = (unsigned)(bk >> 32);
+  const unsigned mhi = __reduce_max_sync(kFull, hi);
+  if (mhi == 0u && __ballot_sync(kFull, bj >= 0) == 0u) return -1;
+  const unsigned lo = (hi == mhi && bj >= 0) ? (unsigned)bk : 0u;
+  const unsigned mlo = __reduce_max_sync(kFull, lo);
+  const unsigned cand = __ballot_sync(kFull, bj >= 0 && hi == mhi && (unsigned)bk == mlo);
+  if (__popc(cand) == 1) return __shfl_sync(kFull, bj, __ffs(cand) - 1);
+  const unsigned t = ((cand >> lane) & 1u) ? K.tie(bj) : 0xffffffffu;
+  const unsigned mt = __reduce_min_sync(kFull, t);
+  const unsigned who = __ballot_sync(kFull, ((cand >> lane) & 1u) && t == mt);
+  return __shfl_sync(kFull, bj, __ffs(who) - 1);
+}
+
+__device__ __forceinline__ int warp_popc(const unsigned* bm, int words, int lane) {
+  int c = 0;
+  for (int w = lane; w < words; w += 32) c += __popc(bm[w]);
+  return __reduce_add_sync(kFull, c);
+}
+
+// Keep exactly the c best blocks of `mask` (in place).  Uses the cheaper of c
+// argmax rounds into `tmp` or (p - c) argmin rounds out of `mask`.
+__device__ void keep_best(unsigned* mask, unsigned* tmp, int words, int c, int lane, Keys K) {
+  const int p = warp_popc(mask, words, lane);
+  if (p <= c) return;
+  const bool drop = (p - c) < c;
+  K.worst = drop;
+  const int rounds = drop ? p - c : c;
+  if (!drop) {
+    for (int w = lane; w < words; w += 32) tmp[w] = 0u;
+    __syncwarp();
+  }
+  unsigned long long bk;
+  int bj;
+  lane_best(mask, words, lane, K, bk, bj);
+  for (int r = 0; r < rounds; ++r) {
+    const int j = warp_winner(bk, bj, K, lane);
+    if (j < 0) break;
+    if ((j & 31) == lane) {
+      mask[j >> 5] &= ~(1u << lane);
+      if (!drop) tmp[j >> 5] |= (1u << lane);
+      lane_best(mask, words, lane, K, bk, bj);
     }
     __syncwarp();
   }
+  if (!drop) {
+    for (int w = lane; w < words; w += 32) mask[w] = tmp[w];
+  }
+  __syncwarp();
 }
 
 // Write the set bits of bm in ascending order to out[0..cap); returns the count.
@@ -110,24 +164,21 @@ __device__ int bitmap_to_list(const unsigned* bm, int words, int* out, int cap, 
   return base;
 }
 
-__device__ __forceinline__ int warp_sum(int x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
-  return x;
-}
-
 __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectArgs a) {
-  extern __shared__ unsigned sm_sel[];
+  extern __shared__ unsigned long long sm_sel64[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * kSelWarps + warp;
   if (blockIdx.x == 0 && threadIdx.x == 0) a.ds->gather_count = 0;
   if (u >= a.U) return;
 
   const int W = a.words;
-  unsigned* bmE = sm_sel + (size_t)warp * 4 * W;  // Gamma_e(t)
-  unsigned* bmP = bmE + W;                         // S(t-1)
-  unsigned* bmX = bmP + W;                         // working candidate set
-  unsigned* bmS = bmX + W;                         // winners / S(t)
+  const bool stage = a.max_blocks <= kSmemKeys;
+  unsigned long long* skeys = sm_sel64 + (size_t)warp * (stage ? a.max_blocks : 0);
+  unsigned* bmE = reinterpret_cast<unsigned*>(sm_sel64 + (size_t)kSelWarps * (stage ? a.max_blocks : 0)) +
+                  (size_t)warp * 4 * W;                 // Gamma_e(t)
+  unsigned* bmP = bmE + W;                             // S(t-1)
+  unsigned* bmX = bmP + W;                             // working set
+  unsigned* bmT = bmX + W;                             // scratch / S(t)
 
   const int n = a.ds->n_closed;
   const int t = a.ds->step;
@@ -135,8 +186,13 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectArgs a) {
   const int n_from = a.ds->n_last_select;
   const int nw = (n + 31) / 32;
 
+  const double* sc = a.scores + (size_t)u * a.max_blocks;
+  const float* ag = a.agnostic + (size_t)u * a.max_blocks;
+  if (stage) {
+    for (int j = lane; j < n; j += 32) skeys[j] = key_f64(sc[j]);
+  }
   for (int w = lane; w < W; w += 32) {
-    bmE[w] = 0u; bmP[w] = 0u; bmX[w] = 0u; bmS[w] = 0u;
+    bmE[w] = 0u; bmP[w] = 0u; bmX[w] = 0u; bmT[w] = 0u;
   }
   __syncwarp();
 
@@ -149,58 +205,50 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectArgs a) {
     }
     for (int i = lane; i < a.k_e; i += 32) {
       const int bj = ge[i];
-      if (bj >= 0 && bj < n) atomicOr(&bmX[bj >> 5], 1u << (bj & 31));
+      if (bj >= 0 && bj < n) atomicOr(&bmE[bj >> 5], 1u << (bj & 31));
     }
   }
   __syncwarp();
-  // pool of Gamma_e: everything at t = 0, else Gamma_e(t-1) ∪ [n_from, n)
-  const int pool_lo = first ? 0 : n_from;
-  for (int w = lane; w < nw; w += 32) {
-    unsigned add = valid_bits(w, n) & ~valid_bits(w, pool_lo);
-    bmX[w] |= add;
+
+  // ---- Gamma_e: unchanged unless this is the first step or blocks closed
+  const Keys KA{nullptr, ag, nullptr, false};
+  const Keys KS{stage ? skeys : nullptr, nullptr, sc, false};
+  if (first || n_from < n) {
+    const int pool_lo = first ? 0 : n_from;
+    for (int w = lane; w < nw; w += 32) bmE[w] |= valid_bits(w, n) & ~valid_bits(w, pool_lo);
+    __syncwarp();
+    keep_best(bmE, bmT, nw, a.k_e, lane, KA);
   }
-  __syncwarp();
 
-  const float* ag = a.agnostic + (size_t)u * a.max_blocks;
-  const double* sc = a.scores + (size_t)u * a.max_blocks;
-  auto key_a = [ag](int j) { return (double)ag[j]; };
-  auto key_s = [sc](int j) { return sc[j]; };
-
-  warp_topk(bmX, bmE, nw, a.k_e, lane, key_a);
-  __syncwarp();
-
+  // ---- Gamma_q
   if (first) {
     for (int w = lane; w < nw; w += 32) bmX[w] = valid_bits(w, n) & ~bmE[w];
+    __syncwarp();
   } else {
     int e_new = 0;
     for (int w = lane; w < nw; w += 32) {
       e_new += __popc(bmE[w] & ~bmP[w]);
       bmX[w] = valid_bits(w, n) & ~bmE[w] & ~bmP[w];  // new candidates
     }
-    e_new = warp_sum(e_new);
+    e_new = __reduce_add_sync(kFull, e_new);
     const int c_t = max(0, a.c_max - e_new);
     __syncwarp();
-    warp_topk(bmX, bmS, nw, c_t, lane, key_s);
+    keep_best(bmX, bmT, nw, c_t, lane, KS);
+    for (int w = lane; w < nw; w += 32) bmX[w] |= bmP[w] & ~bmE[w];  // ∪ old candidates
     __syncwarp();
-    for (int w = lane; w < nw; w += 32) {
-      bmX[w] = (bmP[w] & ~bmE[w]) | bmS[w];
-      bmS[w] = 0u;
-    }
   }
-  __syncwarp();
-  warp_topk(bmX, bmS, nw, a.k_q, lane, key_s);
-  __syncwarp();
+  keep_best(bmX, bmT, nw, a.k_q, lane, KS);
 
   int ov = 0;
   for (int w = lane; w < nw; w += 32) {
-    bmS[w] |= bmE[w];
-    ov += __popc(bmS[w] & bmP[w]);
+    bmX[w] |= bmE[w];  // S(t)
+    ov += __popc(bmX[w] & bmP[w]);
   }
-  ov = warp_sum(ov);
+  ov = __reduce_add_sync(kFull, ov);
   __syncwarp();
 
   int* sel = a.sel + (size_t)u * a.k;
-  const int ns = bitmap_to_list(bmS, nw, sel, a.k, lane);
+  const int ns = bitmap_to_list(bmX, nw, sel, a.k, lane);
   __syncwarp();
   for (int i = lane; i < a.k; i += 32) {
     const int v = i < ns ? sel[i] : -1;
@@ -222,7 +270,9 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectArgs a) {
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   const int grid = (a.U + kSelWarps - 1) / kSelWarps;
-  const size_t smem = (size_t)kSelWarps * 4 * a.words * sizeof(unsigned);
+  const bool stage = a.max_blocks <= kSmemKeys;
+  const size_t smem = (size_t)kSelWarps * ((stage ? a.max_blocks * sizeof(unsigned long long) : 0) +
+                                           4 * a.words * sizeof(unsigned));
   select_kernel<<<grid, kSelWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
