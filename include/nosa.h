@@ -187,6 +187,31 @@ NOSA_API nosa_status nosa_fetch_missing(nosa_ctx* ctx, const int32_t* sel, int32
 NOSA_API nosa_status nosa_sparse_decode(nosa_ctx* ctx, const void* q, const int32_t* sel, void* out,
                                nosa_stream_t stream);
 
+/* Allocation-free variant of the attention step (no counterpart on the
+ * pages: it exists for embedders).  Some callers cannot call cudaMalloc: a
+ * serving engine that reserves nearly all of HBM for its own pool allocator
+ * leaves no room for a library's private buffers, and code that must not add
+ * device-wide synchronisation (cudaMalloc / cudaFree may synchronise) cannot
+ * create a context.  This call needs no context and allocates nothing.
+ *
+ * It computes what nosa_sparse_decode computes for resident KV without a tail:
+ * for each query head h of unit u, out_h = softmax(q_h K^T / sqrt(d)) V over the
+ * 64 tokens of each block listed in sel[u].  q: device bf16 [B, H_q, 128];
+ * k, v: device bf16 [U, max_blocks*64, 128], 16-byte aligned; sel: device
+ * int32 [U, k_sel] of valid block ids (an out-of-range id reads block 0);
+ * out: device bf16 [B, H_q, 128].  Split-KV partials live in a fixed array
+ * inside the library (8.5 MB per GPU that loads it, held until exit): the call
+ * returns NOSA_ERR_INVALID when B*H_kv*ceil(k_sel/4)*G exceeds 16384 rows.
+ * The first call on a device resolves that array's device address (once per
+ * device, with the device current), so make it before any stream capture.
+ * Every call shares the array and leaves its contents behind; each call
+ * clears the small status word it needs and fully writes the partials it
+ * reads, but calls that overlap on the GPU (on different streams) race. */
+NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, const void* v, int batch,
+                                                int n_q_heads, int n_kv_heads, int max_blocks,
+                                                const int32_t* sel, int k_sel, void* out,
+                                                nosa_stream_t stream);
+
 /* Synchronous.  Copies the running totals into *stats. */
 NOSA_API nosa_status nosa_get_stats(nosa_ctx* ctx, nosa_stats* stats);
 

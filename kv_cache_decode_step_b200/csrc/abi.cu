@@ -48,6 +48,8 @@ enum Phase { kReady = 0, kScored = 1, kSelected = 2, kFetched = 3 };
 
 }  // namespace
 
+void nosa::record_error(const char* msg) { g_err = msg ? msg : ""; }
+
 struct nosa_ctx {
   nosa_config cfg{};
   int U = 0, G = 0, k = 0, C = 0, max_blocks = 0, words = 0, device = 0;

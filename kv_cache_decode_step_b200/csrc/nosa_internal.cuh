@@ -287,6 +287,8 @@ struct CloseArgs {
 cudaError_t launch_close(const CloseArgs& a, cudaStream_t st);
 
 cudaError_t launch_advance(DevState* ds, DevStats* st, cudaStream_t s);
+// Sets the calling thread's nosa_last_error() message.
+void record_error(const char* msg);
 cudaError_t launch_init_state(DevState* ds, int n_closed, int tail_len, int step, int n_last_select,
                               cudaStream_t s);
 cudaError_t launch_reset_stats(DevStats* st, cudaStream_t s);

@@ -30,7 +30,7 @@ ENTRY_POINTS = (
     "nosa_create", "nosa_destroy", "nosa_attach_kv", "nosa_append_token", "nosa_score_blocks",
     "nosa_select", "nosa_fetch_missing", "nosa_sparse_decode", "nosa_get_stats", "nosa_reset_stats",
     "nosa_check_errors", "nosa_read_cache_map", "nosa_get_state", "nosa_set_state",
-    "nosa_debug_wait_flag", "nosa_last_error", "nosa_version",
+    "nosa_debug_wait_flag", "nosa_last_error", "nosa_version", "nosa_sparse_decode_noalloc",
 )
 
 
@@ -90,6 +90,7 @@ def lib() -> C.CDLL:
             "nosa_debug_wait_flag": ([vp, vp, i32, vp], st),
             "nosa_last_error": ([], C.c_char_p),
             "nosa_version": ([], C.c_char_p),
+            "nosa_sparse_decode_noalloc": ([vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp], st),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -209,6 +210,13 @@ def nosa_set_state(ctx, blob: bytes) -> None:
 def nosa_debug_wait_flag(ctx, flag, timeout_ms: int, stream=None) -> None:
     _check(lib().nosa_debug_wait_flag(ctx, _ptr(flag), int(timeout_ms), _stream(stream)),
            "nosa_debug_wait_flag")
+
+
+def nosa_sparse_decode_noalloc(q, k, v, batch: int, n_q_heads: int, n_kv_heads: int, max_blocks: int,
+                               sel, k_sel: int, out, stream=None) -> None:
+    _check(lib().nosa_sparse_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), int(batch), int(n_q_heads),
+                                            int(n_kv_heads), int(max_blocks), _ptr(sel), int(k_sel),
+                                            _ptr(out), _stream(stream)), "nosa_sparse_decode_noalloc")
 
 
 def config_from_workload(w) -> nosa_config:
