@@ -327,7 +327,9 @@ def run_ours(args):
     # ---- end to end through host buffers: q from pinned host, out to pinned host
     e2e = e2e_pass(torch, dec, w, nosa, args.e2e_steps)
 
-    launches_per_step = 8  # score, select, plan, gather, attend x2, combine, advance
+    # kernels per step: score, select, [plan, gather], attention hits pass,
+    # [misses pass + merge | combine], advance, [append, close]
+    launches_per_step = (7 if w.offloaded else 5) + (2 if w.append else 0)
     gather_ms = phase["gather_ms"]
     attn_ms = phase["attention_ms"]
     gather_gbs = (phase["fetched_bytes_per_step"] / (gather_ms * 1e-3) / 1e9) if gather_ms > 0 else 0.0
@@ -400,6 +402,8 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
     ev = {k: torch.cuda.Event(enable_timing=True, external=True) for k in ("a", "b", "c", "d", "g", "e")}
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
+        if w.append:
+            nosa.nosa_append_token(dec.ctx, dec.k_in, dec.v_in, dec.a_in, s)
         ev["a"].record(s)
         nosa.nosa_score_blocks(dec.ctx, dec.q, dec.scores, s)
         ev["b"].record(s)
@@ -420,7 +424,7 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
     for _ in range(n):
         t = dec.t
         with torch.cuda.stream(s):
-            dec.q.copy_(dec.q_all[t], non_blocking=True)
+            dec._load_inputs(t)
             g.replay()
         dec.t += 1
         torch.cuda.synchronize()
@@ -453,7 +457,11 @@ def e2e_pass(torch, dec, w, nosa, n):
         t = dec.t
         with torch.cuda.stream(s):
             dec.q.copy_(q_host[t], non_blocking=True)
-            dec._calls(None)
+            if w.append:
+                dec.k_in.copy_(dec.k_new[t], non_blocking=True)
+                dec.v_in.copy_(dec.v_new[t], non_blocking=True)
+                dec.a_in.copy_(dec.a_new[t], non_blocking=True)
+            dec._calls(w.append)
             out_host.copy_(dec.out, non_blocking=True)
         s.synchronize()
         dec.t += 1

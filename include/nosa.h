@@ -201,7 +201,7 @@ NOSA_API nosa_status nosa_sparse_decode(nosa_ctx* ctx, const void* q, const int3
  * int32 [U, k_sel] of valid block ids (an out-of-range id reads block 0);
  * out: device bf16 [B, H_q, 128].  Split-KV partials live in a fixed array
  * inside the library (8.5 MB per GPU that loads it, held until exit): the call
- * returns NOSA_ERR_INVALID when B*H_kv*ceil(k_sel/4)*G exceeds 16384 rows.
+ * returns NOSA_ERR_INVALID when B*H_q exceeds 8192 query heads.
  * The first call on a device resolves that array's device address (once per
  * device, with the device current), so make it before any stream capture.
  * Every call shares the array and leaves its contents behind; each call

@@ -93,7 +93,8 @@ struct nosa_ctx {
   bool h_appended = false, appends_enabled = false;
   Phase phase = kReady;
 
-  int bps = 4, S1 = 1, S2 = 0, nparts = 2, gather_grid = 148;
+  int nparts = 2, gather_grid = 148, attn_grid = 296;
+  int* unit_done = nullptr;
 };
 
 namespace {
@@ -173,7 +174,7 @@ void free_all(nosa_ctx* c) {
   void* ptrs[] = {c->kbar,   c->agnostic,   c->ge,        c->prev,   c->cache_k,   c->cache_v,
                   c->slot_block, c->last_used, c->block_slot, c->items, c->n_hit,   c->n_items,
                   c->glist,  c->tail_k,     c->tail_v,    c->a_pending, c->part_o, c->part_ml,
-                  c->ds,     c->st,         c->refill_count};
+                  c->ds,     c->st,         c->refill_count, c->unit_done};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (c->ev_plan) cudaEventDestroy(c->ev_plan);
@@ -239,14 +240,19 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
     delete c;
     return fail(NOSA_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
   }
-  if (const char* v = getenv("NOSA_BLOCKS_PER_SPLIT")) c->bps = atoi(v) > 0 ? atoi(v) : 4;
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device);
-  c->gather_grid = sms;
-  if (const char* v = getenv("NOSA_GATHER_CTAS")) c->gather_grid = atoi(v) > 0 ? atoi(v) : sms;
-  c->S1 = (c->k + c->bps - 1) / c->bps;
-  c->S2 = c->offloaded ? 1 : 0;
-  c->nparts = c->S1 + 1;
+  // a quarter of the SMs keeps ~1 MiB of PCIe reads in flight, well past the
+  // link's bandwidth-delay product; more CTAs only queue system-memory
+  // requests that slow the attention running beside the gather
+  c->gather_grid = (sms + 3) / 4;
+  if (const char* v = getenv("NOSA_GATHER_CTAS")) c->gather_grid = atoi(v) > 0 ? atoi(v) : c->gather_grid;
+  // two persistent attention CTAs per SM, each over an equal share of the
+  // (unit, block) positions; a unit's blocks span a few CTAs' shares
+  int want = 2 * sms;
+  if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
+  c->attn_grid = attend_hits_grid(c->U, c->k, 1, want);
+  c->nparts = attend_hits_parts(c->U, c->k, 1, c->attn_grid);
 
   const size_t U = c->U, MB = c->max_blocks, K = c->k;
 #define ALLOC(ptr, n)                    \
@@ -270,6 +276,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   ALLOC(c->ds, 1);
   ALLOC(c->st, 1);
   ALLOC(c->refill_count, 1);
+  ALLOC(c->unit_done, U);
   ALLOC(c->n_hit, U);
   ALLOC(c->n_items, U);
   ALLOC(c->items, U * K);
@@ -291,6 +298,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   if (cudaMemset(c->tail_k, 0, U * kP * kD * 2) != cudaSuccess ||
       cudaMemset(c->tail_v, 0, U * kP * kD * 2) != cudaSuccess ||
       cudaMemset(c->a_pending, 0, U * sizeof(float)) != cudaSuccess ||
+      cudaMemset(c->unit_done, 0, U * sizeof(int)) != cudaSuccess ||
       cudaMemset(c->ds, 0, sizeof(DevState)) != cudaSuccess)
     return cleanup(fail(NOSA_ERR_CUDA, "cudaMemset failed"));
   if (cudaEventCreateWithFlags(&c->ev_plan, cudaEventDisableTiming) != cudaSuccess ||
@@ -540,38 +548,22 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
   a.max_blocks = c->max_blocks;
   a.C = c->C;
   a.resident = c->offloaded ? 0 : 1;
-  a.bps = c->bps;
-  a.nparts = c->nparts;
-  // phase 1: blocks already resident (hits, or everything when KV is in HBM)
-  // plus the open tail; may overlap the gather running on the copy stream
-  a.phase = 1;
-  a.splits = c->S1;
-  a.part_base = 0;
   a.tail_split = 1;
-  NOSA_CUDA(launch_decode(a, c->maps, st));
+  a.nparts = c->nparts;
+  a.part_base = 0;
+  a.hits_grid = c->attn_grid;
+  a.out = static_cast<uint16_t*>(out);
+  // hits pass: blocks already on the GPU (all of S(t) when KV is in HBM) plus
+  // the open tail; it overlaps the gather running on the copy stream.  With
+  // KV in HBM the last CTA of each unit writes the output.
+  a.unit_done = c->offloaded ? nullptr : c->unit_done;
+  NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st));
   if (c->offloaded) {
-    // phase 2: one CTA per unit attends to its fetched blocks once the gather
-    // has landed and merges every partial of the unit into the output
+    // misses pass: one CTA per unit attends to the fetched blocks once the
+    // gather has landed and merges every partial of the unit into the output
     if (c->gather_on_side) NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
-    a.phase = 2;
-    a.splits = 1;
-    a.part_base = c->S1 + 1;
-    a.tail_split = 0;
-    a.merge_out = 1;
-    a.out = static_cast<uint16_t*>(out);
-    NOSA_CUDA(launch_decode(a, c->maps, st));
-  } else {
-    CombineArgs cb{};
-    cb.part_o = c->part_o;
-    cb.part_ml = c->part_ml;
-    cb.out = static_cast<uint16_t*>(out);
-    cb.ds = c->ds;
-    cb.U = c->U;
-    cb.Hq = c->cfg.n_q_heads;
-    cb.Hkv = c->cfg.n_kv_heads;
-    cb.G = c->G;
-    cb.nparts = c->nparts;
-    NOSA_CUDA(launch_combine(cb, st));
+    a.unit_done = nullptr;
+    NOSA_CUDA(launch_attend_misses(a, c->maps, st));
   }
   if (c->appends_enabled) {
     CloseArgs cl{};

@@ -21,8 +21,11 @@
 namespace nosa {
 
 // Capacity of the shared scratch: partial rows of (128 fp32 accumulators) plus
-// one (max, sum) pair each.  A call needs U * ceil(k / 4) * G rows.
+// one (max, sum) pair each, and one merge counter per unit.  A call with U
+// units of G query heads needs U * G * (ceil(grid / U) + 1) rows for a grid of
+// at most 2 CTAs per SM; that fits whenever U * G = B * H_q <= kNoAllocHeads.
 constexpr int kNoAllocRows = 16384;
+constexpr int kNoAllocHeads = 8192;
 
 // File-scope scratch, held by every GPU that loads the library until exit.
 // Host code must not use these names as device addresses; it takes their
@@ -30,10 +33,10 @@ constexpr int kNoAllocRows = 16384;
 static __device__ __align__(256) float g_noalloc_part_o[kNoAllocRows * kD];
 static __device__ __align__(256) float2 g_noalloc_part_ml[kNoAllocRows];
 static __device__ __align__(256) DevState g_noalloc_state;
+static __device__ __align__(256) int g_noalloc_unit_done[kNoAllocRows];
 
 namespace {
 
-constexpr int kNoAllocBlocksPerSplit = 4;
 constexpr int kMaxDevices = 64;
 
 struct DeviceScratch {
@@ -41,6 +44,7 @@ struct DeviceScratch {
   float* part_o = nullptr;
   float2* part_ml = nullptr;
   DevState* state = nullptr;
+  int* unit_done = nullptr;
 };
 
 DeviceScratch g_dev[kMaxDevices];
@@ -74,6 +78,9 @@ nosa_status device_scratch(int dev, DeviceScratch** out) {
     e = cudaGetSymbolAddress(&p, g_noalloc_state);
     if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     d.state = static_cast<DevState*>(p);
+    e = cudaGetSymbolAddress(&p, g_noalloc_unit_done);
+    if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    d.unit_done = static_cast<int*>(p);
     e = configure_decode();
     if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "kernel configuration: %s", cudaGetErrorString(e));
     d.ready = true;
@@ -125,13 +132,10 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
     return noalloc_fail(NOSA_ERR_INVALID, "need 1 <= k_sel <= max_blocks");
   const long long U = (long long)batch * n_kv_heads;
   if (U * max_blocks * kP >= (1ll << 31)) return noalloc_fail(NOSA_ERR_INVALID, "KV rows exceed 2^31");
-  const int splits = (k_sel + kNoAllocBlocksPerSplit - 1) / kNoAllocBlocksPerSplit;
-  const long long rows = U * splits * G;
-  if (rows > kNoAllocRows)
+  if (U * G > kNoAllocHeads)
     return noalloc_fail(NOSA_ERR_INVALID,
-                        "batch x kv_heads x ceil(k/4) x group = %lld partial rows exceeds the fixed scratch "
-                        "of %d rows",
-                        rows, kNoAllocRows);
+                        "batch x n_q_heads = %lld exceeds the %d query heads the fixed scratch holds", U * G,
+                        kNoAllocHeads);
   if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) % 16 != 0)
     return noalloc_fail(NOSA_ERR_INVALID, "K/V base addresses must be 16-byte aligned");
 
@@ -142,14 +146,25 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
   nosa_status s = device_scratch(dev, &ds);
   if (s != NOSA_OK) return s;
 
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = attend_hits_grid((int)U, k_sel, 0, 2 * sms);
+  const int nparts = attend_hits_parts((int)U, k_sel, 0, grid);
+  if (U * nparts * G > kNoAllocRows)
+    return noalloc_fail(NOSA_ERR_INVALID, "%lld partial rows exceed the fixed scratch of %d rows",
+                        U * nparts * G, kNoAllocRows);
+
   DecodeMaps maps{};
   if ((s = encode_rows(&maps.k, k, (unsigned long long)U * max_blocks * kP)) != NOSA_OK) return s;
   if ((s = encode_rows(&maps.v, v, (unsigned long long)U * max_blocks * kP)) != NOSA_OK) return s;
-  maps.tk = maps.k;  // no tail split is launched
+  maps.tk = maps.k;  // there is no tail item
   maps.tv = maps.v;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   e = cudaMemsetAsync(ds->state, 0, sizeof(DevState), st);
+  if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+
+  e = cudaMemsetAsync(ds->unit_done, 0, (size_t)U * sizeof(int), st);
   if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
 
   DecodeArgs a{};
@@ -165,27 +180,14 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
   a.k = k_sel;
   a.max_blocks = max_blocks;
   a.resident = 1;
-  a.phase = 1;
-  a.splits = splits;
-  a.bps = kNoAllocBlocksPerSplit;
-  a.part_base = 0;
-  a.nparts = splits;
   a.tail_split = 0;
-  e = launch_decode(a, maps, st);
+  a.part_base = 0;
+  a.nparts = nparts;
+  a.hits_grid = grid;
+  a.unit_done = ds->unit_done;
+  a.out = static_cast<uint16_t*>(out);
+  e = launch_attend_hits(a, maps, grid, st);
   if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
-
-  CombineArgs cb{};
-  cb.part_o = ds->part_o;
-  cb.part_ml = ds->part_ml;
-  cb.out = static_cast<uint16_t*>(out);
-  cb.ds = ds->state;
-  cb.U = (int)U;
-  cb.Hq = n_q_heads;
-  cb.Hkv = n_kv_heads;
-  cb.G = G;
-  cb.nparts = splits;
-  e = launch_combine(cb, st);
-  if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
   return NOSA_OK;
 }
 

@@ -232,7 +232,7 @@ cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t st);
 struct DecodeArgs {
   const uint16_t* q;        // [B, Hq, d]
   const int* sel;           // resident: [U, k] block ids
-  const int* items;         // offloaded: [U, k] slots
+  const int* items;         // offloaded: [U, k] cache slots, hits first
   const int* n_hit;         // [U]
   const int* n_items;       // [U]
   float* part_o;            // [U, nparts, G, d]
@@ -240,26 +240,26 @@ struct DecodeArgs {
   DevState* ds;
   int U, Hq, Hkv, G, k, max_blocks, C;
   int resident;             // 1: sel indexes the resident KV
-  int phase;                // 1: hits (+ tail split), 2: misses
-  int splits, bps, part_base, nparts, tail_split;
-  int merge_out;            // 1: one CTA per unit, merge parts [0, part_base) and write out
-  uint16_t* out;            // [B, Hq, d] when merge_out
+  int tail_split;           // 1: each unit's open tail is attended in the hits pass
+  int part_base, nparts;    // hits pass writes slots part_base + segment; nparts per unit
+  int hits_grid;            // CTAs of the hits pass (fixes each unit's segment count)
+  int* unit_done;           // resident: per-unit counters, the last CTA merges (else null)
+  uint16_t* out;            // [B, Hq, d]
 };
 struct DecodeMaps {
   CUtensorMap k, v;         // main K/V: resident KV or the cache, rows of 128 bf16
   CUtensorMap tk, tv;       // open tail blocks
 };
-cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st);
+// Hits pass (persistent, `grid` CTAs, which must equal a.hits_grid); partials,
+// and with unit_done the output.
+cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st);
+// The hits-pass grid for a requested CTA count (at most one CTA per position).
+int attend_hits_grid(int U, int k, int tail_split, int want);
+// Partial slots per unit the hits pass writes for this shape and requested grid.
+int attend_hits_parts(int U, int k, int tail_split, int want);
+// Misses pass: one CTA per unit, merges parts [0, part_base) into out.
+cudaError_t launch_attend_misses(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st);
 cudaError_t configure_decode();
-
-struct CombineArgs {
-  const float* part_o;
-  const float2* part_ml;
-  uint16_t* out;            // [B, Hq, d]
-  DevState* ds;
-  int U, Hq, Hkv, G, nparts;
-};
-cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 
 struct AppendArgs {
   const uint16_t* k_new;    // [B, Hkv, d]

@@ -65,6 +65,10 @@ class Decoder:
                 if (tok + 1) % w.block == 0:
                     a_new[t] = data["a"][:, tok // w.block]
             self.a_new = torch.from_numpy(a_new).to(self.dev)
+            # static per-step inputs of the append call (graph replays read these)
+            self.k_in = torch.empty_like(self.k_new[0])
+            self.v_in = torch.empty_like(self.v_new[0])
+            self.a_in = torch.empty_like(self.a_new[0])
         self.q = torch.empty((w.batch, w.n_q_heads, d), dtype=torch.bfloat16, device=self.dev)
         self.scores = torch.zeros((U, w.max_blocks), dtype=torch.float64, device=self.dev)
         self.sel = torch.zeros((U, w.k), dtype=torch.int32, device=self.dev)
@@ -102,11 +106,18 @@ class Decoder:
             pass
 
     # ------------------------------------------------------------ one step
-    def _calls(self, t_append: Optional[int]) -> None:
+    def _load_inputs(self, t: int) -> None:
+        """Copy step t's inputs into the static buffers (on self.stream)."""
+        self.q.copy_(self.q_all[t], non_blocking=True)
+        if self.w.append:
+            self.k_in.copy_(self.k_new[t], non_blocking=True)
+            self.v_in.copy_(self.v_new[t], non_blocking=True)
+            self.a_in.copy_(self.a_new[t], non_blocking=True)
+
+    def _calls(self, append: bool) -> None:
         s, cs = self.stream, self.copy_stream
-        if t_append is not None:
-            nosa.nosa_append_token(self.ctx, self.k_new[t_append], self.v_new[t_append],
-                                   self.a_new[t_append], s)
+        if append:
+            nosa.nosa_append_token(self.ctx, self.k_in, self.v_in, self.a_in, s)
         nosa.nosa_score_blocks(self.ctx, self.q, self.scores, s)
         nosa.nosa_select(self.ctx, self.scores, self.sel, s)
         nosa.nosa_fetch_missing(self.ctx, self.sel, self.fetch, self.n_fetch, s, cs)
@@ -116,23 +127,23 @@ class Decoder:
         """Eager step t (queries of step t copied into the static q buffer)."""
         t = self.t
         with torch.cuda.stream(self.stream):
-            self.q.copy_(self.q_all[t], non_blocking=True)
-            self._calls(t if self.w.append else None)
+            self._load_inputs(t)
+            self._calls(self.w.append)
         self.t += 1
 
     def capture(self) -> None:
-        """Capture one step (without the q copy) in a CUDA graph.  The capture
-        itself enqueues nothing that runs; replays advance the device state."""
-        assert not self.w.append, "graph capture here covers workloads without appends"
+        """Capture one step (without the input copies) in a CUDA graph.  The
+        capture itself runs nothing; replays advance the device-side state
+        (step counter, closed blocks, tail length)."""
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=self.stream):
-            self._calls(None)
+            self._calls(self.w.append)
         self.graph = g
 
     def replay(self) -> None:
         t = self.t
         with torch.cuda.stream(self.stream):
-            self.q.copy_(self.q_all[t], non_blocking=True)
+            self._load_inputs(t)
             self.graph.replay()
         self.t += 1
 

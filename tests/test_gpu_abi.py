@@ -100,8 +100,10 @@ def test_bounded_wait_times_out_and_context_survives(tiny):
         dec.close()
 
 
-def test_graph_replay_equals_eager():
-    w = configs.get("offload_b64", batch=8, steps=10)
+@pytest.mark.parametrize("name,kw", [("offload_b64", {"batch": 8, "steps": 10}),
+                                     ("tiny", {"steps": 80, "append": True, "context": 4096 + 20})])
+def test_graph_replay_equals_eager(name, kw):
+    w = configs.get(name, **kw)
     data = inputs.generate(w)
     outs = []
     for graph in (False, True):

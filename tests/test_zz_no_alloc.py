@@ -51,11 +51,11 @@ def test_noalloc_attention_matches_the_context_path_on_two_calls():
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    q = torch.zeros((256, 32, 128), dtype=torch.bfloat16, device="cuda")
-    kv = torch.zeros((8, 64 * 64, 128), dtype=torch.bfloat16, device="cuda")
-    sel = torch.zeros((256 * 8, 64), dtype=torch.int32, device="cuda")
-    # 256 sequences x 8 KV heads x 16 splits x 4 heads = 131072 rows > 16384
+    q = torch.zeros((512, 32, 128), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((8, 16 * 64, 128), dtype=torch.bfloat16, device="cuda")
+    sel = torch.zeros((512 * 8, 16), dtype=torch.int32, device="cuda")
+    # 512 sequences x 32 query heads = 16384 > 8192: rejected before any launch
     with pytest.raises(nosa.NosaError) as e:
-        nosa.nosa_sparse_decode_noalloc(q, kv, kv, 256, 32, 8, 64, sel, 64, q, None)
+        nosa.nosa_sparse_decode_noalloc(q, kv, kv, 512, 32, 8, 16, sel, 16, q, None)
     assert e.value.status == nosa.NOSA_ERR_INVALID
-    assert "16384" in str(e.value)
+    assert "8192" in str(e.value)
