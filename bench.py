@@ -327,9 +327,10 @@ def run_ours(args):
     # ---- end to end through host buffers: q from pinned host, out to pinned host
     e2e = e2e_pass(torch, dec, w, nosa, args.e2e_steps)
 
-    # kernels per step: score, select, [plan, gather], attention hits pass,
-    # [misses pass + merge | combine], advance, [append, close]
-    launches_per_step = (7 if w.offloaded else 5) + (2 if w.append else 0)
+    # kernels per step: score, select, [plan, gather, misses pass], hits pass;
+    # with appends also append, close and advance (otherwise the last
+    # attention CTA ends the step)
+    launches_per_step = (6 if w.offloaded else 3) + (3 if w.append else 0)
     gather_ms = phase["gather_ms"]
     attn_ms = phase["attention_ms"]
     gather_gbs = (phase["fetched_bytes_per_step"] / (gather_ms * 1e-3) / 1e9) if gather_ms > 0 else 0.0

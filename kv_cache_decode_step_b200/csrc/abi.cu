@@ -95,6 +95,7 @@ struct nosa_ctx {
 
   int nparts = 2, gather_grid = 148, attn_grid = 296;
   int* unit_done = nullptr;
+  int* done_ctr = nullptr;
 };
 
 namespace {
@@ -174,7 +175,7 @@ void free_all(nosa_ctx* c) {
   void* ptrs[] = {c->kbar,   c->agnostic,   c->ge,        c->prev,   c->cache_k,   c->cache_v,
                   c->slot_block, c->last_used, c->block_slot, c->items, c->n_hit,   c->n_items,
                   c->glist,  c->tail_k,     c->tail_v,    c->a_pending, c->part_o, c->part_ml,
-                  c->ds,     c->st,         c->refill_count, c->unit_done};
+                  c->ds,     c->st,         c->refill_count, c->unit_done, c->done_ctr};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (c->ev_plan) cudaEventDestroy(c->ev_plan);
@@ -277,6 +278,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   ALLOC(c->st, 1);
   ALLOC(c->refill_count, 1);
   ALLOC(c->unit_done, U);
+  ALLOC(c->done_ctr, 1);
   ALLOC(c->n_hit, U);
   ALLOC(c->n_items, U);
   ALLOC(c->items, U * K);
@@ -299,6 +301,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
       cudaMemset(c->tail_v, 0, U * kP * kD * 2) != cudaSuccess ||
       cudaMemset(c->a_pending, 0, U * sizeof(float)) != cudaSuccess ||
       cudaMemset(c->unit_done, 0, U * sizeof(int)) != cudaSuccess ||
+      cudaMemset(c->done_ctr, 0, sizeof(int)) != cudaSuccess ||
       cudaMemset(c->ds, 0, sizeof(DevState)) != cudaSuccess)
     return cleanup(fail(NOSA_ERR_CUDA, "cudaMemset failed"));
   if (cudaEventCreateWithFlags(&c->ev_plan, cudaEventDisableTiming) != cudaSuccess ||
@@ -380,6 +383,8 @@ nosa_status nosa_attach_kv(nosa_ctx* c, const void* k, const void* v, int n_toke
   }
   if ((s = reset_tables(c, st)) != NOSA_OK) return s;
   NOSA_CUDA(launch_init_state(c->ds, n, tail, 0, 0, st));
+  NOSA_CUDA(cudaMemsetAsync(c->done_ctr, 0, sizeof(int), st));
+  NOSA_CUDA(cudaMemsetAsync(c->unit_done, 0, U * sizeof(int), st));
   NOSA_CUDA(launch_reset_stats(c->st, st));
   c->attached = true;
   c->h_n_closed = n;
@@ -553,16 +558,22 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
   a.part_base = 0;
   a.hits_grid = c->attn_grid;
   a.out = static_cast<uint16_t*>(out);
+  a.st = c->st;
+  // Without a block close to follow, the last CTA of the step's last kernel
+  // ends the step itself (one launch fewer).
+  const bool fold_advance = !c->appends_enabled;
   // hits pass: blocks already on the GPU (all of S(t) when KV is in HBM) plus
   // the open tail; it overlaps the gather running on the copy stream.  With
   // KV in HBM the last CTA of each unit writes the output.
   a.unit_done = c->offloaded ? nullptr : c->unit_done;
+  a.done_ctr = (fold_advance && !c->offloaded) ? c->done_ctr : nullptr;
   NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st));
   if (c->offloaded) {
     // misses pass: one CTA per unit attends to the fetched blocks once the
     // gather has landed and merges every partial of the unit into the output
     if (c->gather_on_side) NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
     a.unit_done = nullptr;
+    a.done_ctr = fold_advance ? c->done_ctr : nullptr;
     NOSA_CUDA(launch_attend_misses(a, c->maps, st));
   }
   if (c->appends_enabled) {
@@ -579,7 +590,7 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
     cl.max_blocks = c->max_blocks;
     NOSA_CUDA(launch_close(cl, st));
   }
-  NOSA_CUDA(launch_advance(c->ds, c->st, st));
+  if (!fold_advance) NOSA_CUDA(launch_advance(c->ds, c->st, st));
   if (c->h_tail >= kP) {
     c->h_n_closed += 1;
     c->h_tail = 0;

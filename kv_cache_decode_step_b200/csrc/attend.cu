@@ -36,6 +36,12 @@ constexpr int kStageBytes = 2 * kBlockBytes;
 constexpr int kBarOffset = kStages * kStageBytes;
 constexpr int kFlagOffset = kBarOffset + kStages * 8;
 constexpr int kSmemBytes = kFlagOffset + 16 + 1024;  // + slack for 1024-byte alignment
+// The misses pass holds one block at a time (a unit misses 0-3 blocks in the
+// steady state), so six of its CTAs fit per SM and the whole batch runs in one
+// wave; its warp states reuse the single stage.
+constexpr int kMissStages = 1;
+constexpr int kMissBarOffset = kMissStages * kStageBytes;
+constexpr int kMissSmemBytes = kMissBarOffset + 16 + 1024;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kScoreScale = 0.088388347648318440f * 1.4426950408889634f;  // log2(e) / sqrt(128)
 
@@ -178,41 +184,79 @@ __device__ __forceinline__ void store_partial(const WarpStates& ws, int G, float
   }
 }
 
+// Running log-sum-exp merge of (max m, sum l, accumulator o) triples.
+struct LseMerge {
+  float M = -INFINITY, num = 0.f, den = 0.f;
+  __device__ __forceinline__ void add(float m, float l, float o) {
+    if (!(l > 0.f)) return;
+    if (m > M) {
+      const float s = exp2f(M - m);  // M = -inf gives 0
+      num *= s;
+      den *= s;
+      M = m;
+    }
+    const float f = exp2f(m - M);
+    num += f * o;
+    den += f * l;
+  }
+};
+
 // out[b, g*G + h, :] = merge of the unit's partials [0, nparts) (read around
-// L1: other CTAs wrote them) and, optionally, this CTA's warp states.
+// L1: other CTAs wrote them) and, optionally, this CTA's warp states.  Thread
+// d owns dim d; heads go two at a time, with the loads of four parts of both
+// issued together.
 __device__ void merge_unit(const DecodeArgs& a, int u, int nparts, const WarpStates* ws) {
   const int b = u / a.Hkv, g = u % a.Hkv;
   const float* po = a.part_o + (size_t)u * a.nparts * a.G * kD;
   const float2* pml = a.part_ml + (size_t)u * a.nparts * a.G;
-  for (int idx = threadIdx.x; idx < a.G * kD; idx += blockDim.x) {
-    const int h = idx / kD, dd = idx % kD;
-    float M = -INFINITY;
-    for (int p = 0; p < nparts; ++p) M = fmaxf(M, __ldcg(&pml[p * a.G + h]).x);
-    if (ws) {
+  for (int dd = threadIdx.x; dd < kD; dd += blockDim.x) {
+    for (int h0 = 0; h0 < a.G; h0 += 2) {
+      LseMerge mg[2];
+      for (int p0 = 0; p0 < nparts; p0 += 4) {
+        float2 ml[4][2];
+        float ov[4][2];
 #pragma unroll
-      for (int w = 0; w < 4; ++w) M = fmaxf(M, ws->m[w * kMaxG + h]);
-    }
-    const float Mu = M == -INFINITY ? 0.f : M;
-    float num = 0.f, den = 0.f;
-    for (int p = 0; p < nparts; ++p) {
-      const float2 ml = __ldcg(&pml[p * a.G + h]);
-      if (ml.y <= 0.f) continue;
-      const float f = exp2f(ml.x - Mu);
-      num += f * __ldcg(&po[((size_t)p * a.G + h) * kD + dd]);
-      den += f * ml.y;
-    }
-    if (ws) {
+        for (int i = 0; i < 4; ++i) {
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float l = ws->l[w * kMaxG + h];
-        if (l <= 0.f) continue;
-        const float f = exp2f(ws->m[w * kMaxG + h] - Mu);
-        num += f * ws->o[(w * kMaxG + h) * kD + dd];
-        den += f * l;
+          for (int e = 0; e < 2; ++e) {
+            const int h = h0 + e;
+            const bool on = p0 + i < nparts && h < a.G;
+            ml[i][e] = on ? __ldcg(&pml[(p0 + i) * a.G + h]) : make_float2(-INFINITY, 0.f);
+            ov[i][e] = on ? __ldcg(&po[((size_t)(p0 + i) * a.G + h) * kD + dd]) : 0.f;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          mg[0].add(ml[i][0].x, ml[i][0].y, ov[i][0]);
+          mg[1].add(ml[i][1].x, ml[i][1].y, ov[i][1]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int h = h0 + e;
+        if (h >= a.G) break;
+        if (ws) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            mg[e].add(ws->m[w * kMaxG + h], ws->l[w * kMaxG + h], ws->o[(w * kMaxG + h) * kD + dd]);
+        }
+        const float r = mg[e].den > 0.f ? mg[e].num / mg[e].den : 0.f;
+        a.out[((size_t)b * a.Hq + (size_t)g * a.G + h) * kD + dd] = (uint16_t)(pack_bf16x2(r, 0.f) & 0xFFFFu);
       }
     }
-    const float r = den > 0.f ? num / den : 0.f;
-    a.out[((size_t)b * a.Hq + (size_t)g * a.G + h) * kD + dd] = (uint16_t)(pack_bf16x2(r, 0.f) & 0xFFFFu);
+  }
+}
+
+// Every CTA calls this once at its very end: the last one to arrive ends the
+// step (all other CTAs of the kernel are done with the state by then).
+__device__ __forceinline__ void finish_step(const DecodeArgs& a) {
+  if (!a.done_ctr) return;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0 && atomicAdd(a.done_ctr, 1) == (int)(gridDim.x * gridDim.y) - 1) {
+    __threadfence();
+    advance_step(a.ds, a.st);
+    *a.done_ctr = 0;
   }
 }
 
@@ -383,6 +427,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       __syncthreads();
     }
   }
+  finish_step(a);
 }
 
 // Partial slots a unit needs in the hits pass for a grid of `grid` CTAs.
@@ -392,13 +437,13 @@ __host__ __device__ inline int hits_segments_per_unit(int U, int vpu, int grid) 
   return (int)(((long long)vpu * grid + V - 1) / V) + 1;
 }
 
-// One CTA per unit: the blocks fetched this step, then the merge of every
-// partial of the unit into the output.
-__global__ void __launch_bounds__(kAttnThreads, 2)
+// One CTA per unit: the blocks fetched this step (one at a time), then the
+// merge of every partial of the unit into the output.
+__global__ void __launch_bounds__(kAttnThreads)
     attend_misses_kernel(const __grid_constant__ DecodeMaps maps, DecodeArgs a) {
   extern __shared__ unsigned char attn_smem_raw[];
   unsigned char* sm = aligned_smem(attn_smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kBarOffset);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kMissBarOffset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x;
   const int lo = a.n_hit[u], hi = a.n_items[u];
@@ -411,40 +456,39 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   const int n_segs = wk.cta_of((long long)(u + 1) * wk.vpu - 1) - wk.cta_of((long long)u * wk.vpu) + 1;
   if (n == 0) {
     merge_unit(a, u, n_segs, nullptr);
+    finish_step(a);
     return;
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
+    mbar_init(bar, 1);
     fence_mbar_init();
-    for (int i = 0; i < kStages && i < n; ++i) issue_block(maps, a, sm, bars, i, u, lo + i, false);
+    issue_block(maps, a, sm, bar, 0, u, lo, false);
   }
   __syncthreads();
   uint32_t qf[8][2];
   load_query(a, u, lane, qf);
   AttnAcc acc;
   acc_init(acc);
+  const uint32_t kb = smem_u32(sm);
   for (int j = 0; j < n; ++j) {
-    const int st = j % kStages;
-    const bool ok = mbar_wait_bounded(&bars[st], (uint32_t)((j / kStages) & 1), kWaitLimitNs);
+    const bool ok = mbar_wait_bounded(bar, (uint32_t)(j & 1), kWaitLimitNs);
     if (__syncthreads_or(!ok)) {
-      if (threadIdx.x == 0) {
-        atomicOr(&a.ds->error_bits, ERR_TIMEOUT);
-        const int issued = min(n, j + kStages);
-        for (int g2 = j; g2 < issued; ++g2)
-          (void)mbar_wait_bounded(&bars[g2 % kStages], (uint32_t)((g2 / kStages) & 1), kWaitLimitNs);
-      }
+      if (threadIdx.x == 0) atomicOr(&a.ds->error_bits, ERR_TIMEOUT);
       __syncthreads();
       return;
     }
-    const uint32_t kb = smem_u32(sm + st * kStageBytes);
     attend_block(kb, kb + kBlockBytes, warp, lane, kP, qf, acc);
     __syncthreads();
-    if (threadIdx.x == 0 && j + kStages < n) issue_block(maps, a, sm, bars, st, u, lo + j + kStages, false);
+    if (threadIdx.x == 0 && j + 1 < n) {
+      fence_proxy_async_smem();
+      issue_block(maps, a, sm, bar, 0, u, lo + j + 1, false);
+    }
   }
-  // every load has been consumed: stage 0 holds the warp states
+  // every load has been consumed: the stage holds the warp states
   const WarpStates ws(sm);
   publish_warp_state(acc, ws, warp, lane);
   merge_unit(a, u, n_segs, &ws);
+  finish_step(a);
 }
 
 int attend_smem_bytes() { return kSmemBytes; }
@@ -453,7 +497,7 @@ int attend_smem_bytes() { return kSmemBytes; }
 cudaError_t configure_decode() {
   cudaError_t e = cudaFuncSetAttribute(attend_hits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(attend_misses_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  return cudaFuncSetAttribute(attend_misses_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMissSmemBytes);
 }
 
 cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st) {
@@ -472,7 +516,7 @@ int attend_hits_parts(int U, int k, int tail_split, int grid) {
 }
 
 cudaError_t launch_attend_misses(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st) {
-  attend_misses_kernel<<<a.U, kAttnThreads, kSmemBytes, st>>>(m, a);
+  attend_misses_kernel<<<a.U, kAttnThreads, kMissSmemBytes, st>>>(m, a);
   return cudaGetLastError();
 }
 

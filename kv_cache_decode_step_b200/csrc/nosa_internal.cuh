@@ -102,6 +102,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Untiled bulk copy global -> shared (no multicast), completing on an
+// mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -170,6 +180,23 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double x) {
   return sign | static_cast<uint32_t>(bits);
 }
 
+// End of a step: the selection just made saw n_closed blocks; a full tail
+// becomes a closed block; the step counter advances.  Run by one thread after
+// every other kernel of the step has finished reading the state.
+__device__ __forceinline__ void advance_step(DevState* ds, DevStats* st) {
+  ds->n_last_select = ds->n_closed;
+  const int tl = ds->tail_len_step;
+  if (tl >= kP) {
+    ds->n_closed += 1;
+    ds->tail_len = 0;
+  } else {
+    ds->tail_len = tl;
+  }
+  ds->tail_len_step = ds->tail_len;
+  ds->step += 1;
+  st->steps += 1;
+}
+
 // ------------------------------------------------------------------ launches
 // Each returns the launch error (cudaSuccess if queued).
 
@@ -183,7 +210,7 @@ struct ScoreArgs {
   const uint16_t* q;        // [B, Hq, d]
   const uint16_t* kbar;     // [U, max_blocks*R, d]
   double* scores;           // [U, max_blocks]
-  const DevState* ds;
+  DevState* ds;
   int U, Hq, Hkv, G, max_blocks;
 };
 cudaError_t launch_score(const ScoreArgs& a, cudaStream_t st);
@@ -245,6 +272,8 @@ struct DecodeArgs {
   int hits_grid;            // CTAs of the hits pass (fixes each unit's segment count)
   int* unit_done;           // resident: per-unit counters, the last CTA merges (else null)
   uint16_t* out;            // [B, Hq, d]
+  int* done_ctr;            // non-null: the kernel's last CTA ends the step (advance_step)
+  DevStats* st;
 };
 struct DecodeMaps {
   CUtensorMap k, v;         // main K/V: resident KV or the cache, rows of 128 bf16

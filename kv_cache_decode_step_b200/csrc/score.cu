@@ -55,12 +55,20 @@ cudaError_t launch_pool(const uint16_t* src, size_t src_unit_tokens, int U, int 
 }
 
 // ---------------------------------------------------------------- scoring
-// One CTA = one unit x 64 blocks.  Within a block, lanes 8r..8r+7 hold
-// sub-block r and lane 8r+c owns dims [16c, 16c+16).
+// One CTA = one unit x 32 blocks (32 KiB of pooled keys), four warps of 8
+// blocks.  Thread 0 starts four bulk copies of the CTA's pooled keys into
+// shared memory at once (seven CTAs per SM: the whole batch is in flight in
+// one wave) and each warp waits only for its own 8 blocks.  Within a block,
+// lanes 8r..8r+7 hold sub-block r and lane 8r+c owns dims [8c, 8c+8) and
+// [64+8c, 64+8c+8), so every quarter-warp reads 128 contiguous bytes.
 // The group's queries are summed first (fp64, exact for bf16 inputs), so each
 // sub-block score is one 128-term fp64 dot product whose products are exact;
 // only the summation order differs from the definition.
-constexpr int kScoreBlocksPerCta = 64;
+constexpr int kScoreCtaBlocks = 32;
+constexpr int kScoreWarps = 4;
+constexpr int kScoreWarpBlocks = kScoreCtaBlocks / kScoreWarps;
+constexpr int kBlockU4 = kR * kRowU4;  // 16-byte words of pooled keys per block (64)
+constexpr uint64_t kScoreWaitNs = 1000000000ull;
 
 __device__ __forceinline__ double dot16(const uint4& a, const uint4& b, const double* qt) {
   double s = 0.0;
@@ -85,38 +93,38 @@ __device__ __forceinline__ double block_reduce(double s) {
   return o > s ? o : s;
 }
 
-// Each warp owns 8 consecutive blocks (8 KiB of pooled keys) and issues all of
-// their loads before any arithmetic, so every SM keeps tens of KiB in flight.
-constexpr int kScoreBlocksPerWarp = kScoreBlocksPerCta / 8;
-
-__global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreWarps * 32) score_kernel(ScoreArgs a) {
+  __shared__ __align__(128) uint4 skb[kScoreCtaBlocks * kBlockU4];  // 32 KiB
+  __shared__ __align__(8) uint64_t bars[kScoreWarps];
   const int u = blockIdx.y;
   const int n = a.ds->n_closed;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j0 = blockIdx.x * kScoreBlocksPerCta + warp * kScoreBlocksPerWarp;
+  const int j0 = blockIdx.x * kScoreCtaBlocks;
   if (j0 >= n) return;
-  const int r = lane >> 3, c = lane & 7;
-  const int b = u / a.Hkv, g = u % a.Hkv;
-
-  const uint4* kb = reinterpret_cast<const uint4*>(a.kbar) +
-                    ((size_t)u * a.max_blocks * kR + (size_t)j0 * kR + r) * kRowU4 + 2 * c;
-  uint4 x[kScoreBlocksPerWarp][2];
-#pragma unroll
-  for (int i = 0; i < kScoreBlocksPerWarp; ++i) {
-    if (j0 + i < n) {
-      x[i][0] = kb[(size_t)i * kR * kRowU4];
-      x[i][1] = kb[(size_t)i * kR * kRowU4 + 1];
-    } else {
-      x[i][0] = x[i][1] = make_uint4(0, 0, 0, 0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = min(kScoreCtaBlocks, n - j0);
+  const uint4* src = reinterpret_cast<const uint4*>(a.kbar) + ((size_t)u * a.max_blocks + j0) * kBlockU4;
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < kScoreWarps; ++w) mbar_init(&bars[w], 1);
+    fence_mbar_init();
+    for (int w = 0; w < kScoreWarps; ++w) {
+      const int cnt = min(kScoreWarpBlocks, nb - w * kScoreWarpBlocks);
+      if (cnt <= 0) break;
+      const uint32_t bytes = (uint32_t)cnt * kBlockU4 * 16;
+      mbar_arrive_expect_tx(&bars[w], bytes);
+      bulk_load(skb + w * kScoreWarpBlocks * kBlockU4, src + (size_t)w * kScoreWarpBlocks * kBlockU4, bytes,
+                &bars[w]);
     }
   }
+  __syncthreads();
 
+  const int r = lane >> 3, c = lane & 7;
+  const int b = u / a.Hkv, g = u % a.Hkv;
   double qt[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) qt[i] = 0.0;
-  const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + (size_t)g * a.G) * kD) + 2 * c;
+  const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + (size_t)g * a.G) * kD);
   for (int h = 0; h < a.G; ++h) {
-    const uint4 y0 = qrow[h * kRowU4], y1 = qrow[h * kRowU4 + 1];
+    const uint4 y0 = qrow[h * kRowU4 + c], y1 = qrow[h * kRowU4 + 8 + c];
     const uint32_t wv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -125,24 +133,45 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
     }
   }
 
-  double sres[kScoreBlocksPerWarp];
+  const int jw = warp * kScoreWarpBlocks;
+  const int cnt = min(kScoreWarpBlocks, nb - jw);
+  bool timed_out = false;
+  if (cnt > 0) {
+    if (!mbar_wait_bounded(&bars[warp], 0u, kScoreWaitNs)) {
+      timed_out = true;
+    } else {
+      double sres[kScoreWarpBlocks];
 #pragma unroll
-  for (int i = 0; i < kScoreBlocksPerWarp; ++i) sres[i] = dot16(x[i][0], x[i][1], qt);
+      for (int i = 0; i < kScoreWarpBlocks; ++i) {
+        if (i < cnt) {
+          const uint4* row = skb + (jw + i) * kBlockU4 + r * kRowU4;
+          sres[i] = dot16(row[c], row[8 + c], qt);
+        } else {
+          sres[i] = 0.0;
+        }
+      }
 #pragma unroll
-  for (int i = 0; i < kScoreBlocksPerWarp; ++i) sres[i] = block_reduce(sres[i]);
-  if (lane < kScoreBlocksPerWarp) {
-    // lane i writes block j0 + i (all lanes hold every reduced value)
-    double v = sres[0];
+      for (int i = 0; i < kScoreWarpBlocks; ++i) sres[i] = block_reduce(sres[i]);
+      if (lane < cnt) {
+        double v = sres[0];
 #pragma unroll
-    for (int i = 1; i < kScoreBlocksPerWarp; ++i)
-      if (lane == i) v = sres[i];
-    if (j0 + lane < n) a.scores[(size_t)u * a.max_blocks + j0 + lane] = v;
+        for (int i = 1; i < kScoreWarpBlocks; ++i)
+          if (lane == i) v = sres[i];
+        a.scores[(size_t)u * a.max_blocks + j0 + jw + lane] = v;
+      }
+    }
+  }
+  // never leave a bulk copy in flight behind an exiting CTA
+  if (__syncthreads_or(timed_out) && threadIdx.x == 0) {
+    atomicOr(&a.ds->error_bits, ERR_TIMEOUT);
+    for (int w = 0; w < kScoreWarps; ++w)
+      if (w * kScoreWarpBlocks < nb) (void)mbar_wait_bounded(&bars[w], 0u, kScoreWaitNs);
   }
 }
 
 cudaError_t launch_score(const ScoreArgs& a, cudaStream_t st) {
-  dim3 grid((a.max_blocks + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta, a.U);
-  score_kernel<<<grid, 256, 0, st>>>(a);
+  dim3 grid((a.max_blocks + kScoreCtaBlocks - 1) / kScoreCtaBlocks, a.U);
+  score_kernel<<<grid, kScoreWarps * 32, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -15,8 +15,10 @@
 //   Gamma_q(t) = top-k_q by score of (S(t-1) \ Gamma_e(t)) ∪ top-c_t(new)
 //   S(t)       = Gamma_e(t) ∪ Gamma_q(t), ties to the lower block id.
 //
-// Sets are bitmaps in shared memory; lane l owns the blocks j with j % 32 == l
-// (bit l of word j / 32).  Keys are order-preserving integer images of the
+// Lane l owns the blocks j with j % 32 == l.  Up to 1024 blocks their keys sit
+// in registers and sets are per-lane bit masks; beyond that sets are bitmaps
+// in shared memory (bit l of word j / 32) and keys are read from memory.
+// Keys are order-preserving integer images of the
 // scores (larger score -> larger key), so one warp-wide argmax is two
 // redux.sync max steps, a ballot and, only on an exact tie, a redux.sync min
 // over block ids.  Choosing c of a set of p candidates takes min(c, p - c)
@@ -268,8 +270,201 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- register path
+// For n <= 32 * R: lane l holds blocks j = 32 i + l (i < R) -- their keys in
+// registers and set membership as R-bit masks -- so a round of selection is a
+// warp_winner plus an R-step rescan in registers, and lists come out of one
+// ballot per row i.
+
+template <int R>
+__device__ __forceinline__ void lane_best_reg(uint32_t mask, const unsigned long long (&k)[R], bool worst,
+                                              unsigned long long& bk, int& bi) {
+  bk = 0ull;
+  bi = -1;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    if ((mask >> i) & 1u) {
+      const unsigned long long kk = worst ? ~k[i] : k[i];
+      // rows ascend with i: on equal keys keep the first for "best", the last for "worst"
+      if (bi < 0 || kk > bk || (worst && kk == bk)) {
+        bk = kk;
+        bi = i;
+      }
+    }
+  }
+}
+
+// Keep exactly the c best of `mask` (per-lane R-bit masks, whole warp).
+template <int R>
+__device__ void keep_best_reg(uint32_t& mask, int c, const unsigned long long (&k)[R], int lane) {
+  const int p = (int)__reduce_add_sync(kFull, (unsigned)__popc(mask));
+  if (p <= c) return;
+  const bool worst = (p - c) < c;
+  const int rounds = worst ? p - c : c;
+  uint32_t kept = 0u;
+  unsigned long long bk;
+  int bi;
+  lane_best_reg<R>(mask, k, worst, bk, bi);
+  for (int r = 0; r < rounds; ++r) {
+    const unsigned hi = (unsigned)(bk >> 32);
+    const unsigned mhi = __reduce_max_sync(kFull, hi);
+    if (mhi == 0u) break;
+    const unsigned lo = (bi >= 0 && hi == mhi) ? (unsigned)bk : 0u;
+    const unsigned mlo = __reduce_max_sync(kFull, lo);
+    const unsigned cand = __ballot_sync(kFull, bi >= 0 && hi == mhi && (unsigned)bk == mlo);
+    int wl;  // winning lane
+    if (__popc(cand) == 1) {
+      wl = __ffs(cand) - 1;
+    } else {
+      // equal keys: block id 32*bi + lane decides (smaller for best, larger for worst)
+      const unsigned j = (unsigned)(32 * bi + lane);
+      const unsigned t = ((cand >> lane) & 1u) ? (worst ? ~j : j) : 0xffffffffu;
+      const unsigned mt = __reduce_min_sync(kFull, t);
+      wl = __ffs(__ballot_sync(kFull, ((cand >> lane) & 1u) && t == mt)) - 1;
+    }
+    if (lane == wl) {
+      mask &= ~(1u << bi);
+      if (!worst) kept |= 1u << bi;
+      lane_best_reg<R>(mask, k, worst, bk, bi);
+    }
+  }
+  if (!worst) mask = kept;
+}
+
+// Blocks of the per-lane masks, ascending, into out[0..cap); returns the count.
+template <int R>
+__device__ __forceinline__ int write_list_reg(uint32_t mask, int* out, int cap, int lane) {
+  const unsigned lt = (1u << lane) - 1u;
+  int base = 0;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const bool on = (mask >> i) & 1u;
+    const unsigned bal = __ballot_sync(kFull, on);
+    const int pos = base + __popc(bal & lt);
+    if (on && pos < cap) out[pos] = 32 * i + lane;
+    base += __popc(bal);
+  }
+  return base;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kSelWarps * 32) select_reg_kernel(SelectArgs a) {
+  __shared__ unsigned sbm[kSelWarps][2][R];  // S(t-1) and Gamma_e(t-1) as block bitmaps
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * kSelWarps + warp;
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.ds->gather_count = 0;
+  if (u >= a.U) return;
+
+  const int n = a.ds->n_closed;
+  const int t = a.ds->step;
+  const bool first = (t == 0);
+  const int n_from = a.ds->n_last_select;
+  const double* sc = a.scores + (size_t)u * a.max_blocks;
+  const float* ag = a.agnostic + (size_t)u * a.max_blocks;
+  int* prev = a.prev + (size_t)u * a.k;
+  int* ge = a.ge + (size_t)u * a.k_e;
+
+  unsigned long long ks[R];
+  uint32_t valid = 0u, fresh = 0u;  // closed blocks; blocks closed since the last step
+  const int pool_lo = first ? 0 : n_from;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int j = 32 * i + lane;
+    ks[i] = j < n ? key_f64(sc[j]) : 0ull;
+    if (j < n) valid |= 1u << i;
+    if (j < n && j >= pool_lo) fresh |= 1u << i;
+  }
+  for (int i = lane; i < 2 * R; i += 32) (&sbm[warp][0][0])[i] = 0u;
+  __syncwarp();
+  if (!first) {
+    for (int i = lane; i < a.k; i += 32) {
+      const int bj = prev[i];
+      if (bj >= 0 && bj < n) atomicOr(&sbm[warp][0][bj >> 5], 1u << (bj & 31));
+    }
+    for (int i = lane; i < a.k_e; i += 32) {
+      const int bj = ge[i];
+      if (bj >= 0 && bj < n) atomicOr(&sbm[warp][1][bj >> 5], 1u << (bj & 31));
+    }
+  }
+  __syncwarp();
+  uint32_t mP = 0u, mE = 0u;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    mP |= ((sbm[warp][0][i] >> lane) & 1u) << i;
+    mE |= ((sbm[warp][1][i] >> lane) & 1u) << i;
+  }
+
+  // ---- Gamma_e: unchanged unless this is the first step or blocks closed
+  if (__any_sync(kFull, fresh != 0u)) {
+    unsigned long long ka[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int j = 32 * i + lane;
+      ka[i] = j < n ? key_f32(ag[j]) : 0ull;
+    }
+    mE |= fresh;
+    keep_best_reg<R>(mE, a.k_e, ka, lane);
+  }
+
+  // ---- Gamma_q
+  uint32_t mX;
+  if (first) {
+    mX = valid & ~mE;
+  } else {
+    const int e_new = (int)__reduce_add_sync(kFull, (unsigned)__popc(mE & ~mP));
+    const int c_t = max(0, a.c_max - e_new);
+    mX = valid & ~mE & ~mP;  // new candidates
+    keep_best_reg<R>(mX, c_t, ks, lane);
+    mX |= mP & ~mE;          // ∪ old candidates
+  }
+  keep_best_reg<R>(mX, a.k_q, ks, lane);
+  const uint32_t mS = mX | mE;
+  const int ov = (int)__reduce_add_sync(kFull, (unsigned)__popc(mS & mP));
+
+  int* sel = a.sel + (size_t)u * a.k;
+  const int ns = write_list_reg<R>(mS, sel, a.k, lane);
+  write_list_reg<R>(mS, prev, a.k, lane);
+  for (int i = ns + lane; i < a.k; i += 32) {
+    sel[i] = -1;
+    prev[i] = -1;
+  }
+  const int ne = write_list_reg<R>(mE, ge, a.k_e, lane);
+  for (int i = ne + lane; i < a.k_e; i += 32) ge[i] = -1;
+
+  if (lane == 0) {
+    atomicAdd(&a.st->selected, (unsigned long long)ns);
+    if (!first) {
+      atomicAdd(&a.st->overlap_sum, (unsigned long long)ov);
+      atomicAdd(&a.st->overlap_terms, 1ull);
+      atomicMin(&a.st->min_overlap, ov);
+    }
+  }
+}
+
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   const int grid = (a.U + kSelWarps - 1) / kSelWarps;
+  // register path when every block fits in 32 rows per lane
+  const int rows = (a.max_blocks + 31) / 32;
+  if (rows <= 2) {
+    select_reg_kernel<2><<<grid, kSelWarps * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  }
+  if (rows <= 4) {
+    select_reg_kernel<4><<<grid, kSelWarps * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  }
+  if (rows <= 8) {
+    select_reg_kernel<8><<<grid, kSelWarps * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  }
+  if (rows <= 16) {
+    select_reg_kernel<16><<<grid, kSelWarps * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  }
+  if (rows <= 32) {
+    select_reg_kernel<32><<<grid, kSelWarps * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   const bool stage = a.max_blocks <= kSmemKeys;
   const size_t smem = (size_t)kSelWarps * ((stage ? a.max_blocks * sizeof(unsigned long long) : 0) +
                                            4 * a.words * sizeof(unsigned));

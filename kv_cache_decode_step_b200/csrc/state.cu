@@ -86,19 +86,7 @@ cudaError_t launch_close(const CloseArgs& a, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- step state
-__global__ void advance_kernel(DevState* ds, DevStats* st) {
-  ds->n_last_select = ds->n_closed;
-  const int tl = ds->tail_len_step;
-  if (tl >= kP) {
-    ds->n_closed += 1;
-    ds->tail_len = 0;
-  } else {
-    ds->tail_len = tl;
-  }
-  ds->tail_len_step = ds->tail_len;
-  ds->step += 1;
-  st->steps += 1;
-}
+__global__ void advance_kernel(DevState* ds, DevStats* st) { advance_step(ds, st); }
 
 cudaError_t launch_advance(DevState* ds, DevStats* st, cudaStream_t s) {
   advance_kernel<<<1, 1, 0, s>>>(ds, st);
