@@ -41,6 +41,8 @@ class Workload:
     resample_every: int = 0  # queries replaced by fresh N(0,1) every this many steps
     planted_blocks: int = 0  # blocks per unit whose keys are scaled
     planted_scale: float = 1.0
+    sink_blocks: int = 0     # forced: the first closed blocks (attention sink)
+    window_blocks: int = 0   # forced: the last closed blocks (sliding window)
     head_dim: int = 128
     block: int = 64         # P, tokens per block
     sub_block: int = 16     # Q, tokens per pooled sub-block

@@ -46,7 +46,7 @@ class OrcCfg(C.Structure):
     _fields_ = [("G", C.c_int), ("d", C.c_int), ("P", C.c_int), ("Q", C.c_int),
                 ("n0", C.c_int), ("tail0", C.c_int), ("max_blocks", C.c_int),
                 ("k_q", C.c_int), ("k_e", C.c_int), ("m", C.c_int), ("C", C.c_int),
-                ("steps", C.c_int), ("append", C.c_int)]
+                ("steps", C.c_int), ("append", C.c_int), ("sink", C.c_int), ("window", C.c_int)]
 
 
 def lib():
@@ -69,6 +69,11 @@ def lib():
             L.orc_select.argtypes = [vp, C.c_int, vp, C.c_int, vp, C.c_int, C.c_int,
                                      C.c_int, C.c_int, vp]
             L.orc_select.restype = C.c_int
+            L.orc_select_forced.argtypes = [vp, C.c_int, vp, vp, C.c_int, vp, C.c_int, C.c_int,
+                                            C.c_int, C.c_int, vp]
+            L.orc_select_forced.restype = C.c_int
+            L.orc_forced.argtypes = [C.c_int, C.c_int, C.c_int, vp]
+            L.orc_forced.restype = C.c_int
             L.orc_cache_plan.argtypes = [vp, C.c_int, C.c_int, C.c_int, vp, vp, vp, vp]
             L.orc_cache_plan.restype = C.c_int
             L.orc_attend.argtypes = [vp, C.c_int, C.c_int, vp, vp, vp, C.c_int, vp]
@@ -138,6 +143,28 @@ def select(score: np.ndarray, ge: Sequence[int], prev: Sequence[int], first: boo
     return out[:n].copy()
 
 
+def select_forced(score: np.ndarray, forced: Sequence[int], ge: Sequence[int], prev: Sequence[int],
+                  first: bool, k_q: int, c_max: int) -> np.ndarray:
+    """Selection with forced blocks (ids in `forced`)."""
+    score = _c(score, np.float64)
+    n = score.shape[0]
+    fl = np.zeros(n + 1, dtype=np.uint8)
+    for j in forced:
+        fl[int(j)] = 1
+    g = _c(list(ge) or [0], np.int32)
+    p = _c(list(prev) or [0], np.int32)
+    out = np.zeros(n + 1, dtype=np.int32)
+    m = lib().orc_select_forced(_p(score), n, _p(fl), _p(g), len(ge), _p(p), len(prev),
+                                int(bool(first)), k_q, c_max, _p(out))
+    return out[:m].copy()
+
+
+def forced_blocks(n: int, sink: int, window: int) -> np.ndarray:
+    fl = np.zeros(max(n, 1), dtype=np.uint8)
+    lib().orc_forced(n, sink, window, _p(fl))
+    return np.nonzero(fl[:n])[0]
+
+
 class Cache:
     """Per-unit cache bookkeeping state for :func:`cache_plan`."""
 
@@ -185,14 +212,15 @@ class UnitRun:
     scores: Optional[np.ndarray]    # [steps, max_blocks]
 
 
-def make_cfg(G, d, P, Q, n0, tail0, max_blocks, k_q, k_e, m, C_slots, steps, append) -> OrcCfg:
-    return OrcCfg(G, d, P, Q, n0, tail0, max_blocks, k_q, k_e, m, C_slots, steps, int(append))
+def make_cfg(G, d, P, Q, n0, tail0, max_blocks, k_q, k_e, m, C_slots, steps, append, sink=0,
+             window=0) -> OrcCfg:
+    return OrcCfg(G, d, P, Q, n0, tail0, max_blocks, k_q, k_e, m, C_slots, steps, int(append), sink, window)
 
 
 def cfg_from_workload(w, steps: Optional[int] = None) -> OrcCfg:
     return make_cfg(w.group, w.head_dim, w.block, w.sub_block, w.n_blocks0, w.tail0,
                     w.max_blocks, w.k_query, w.k_agnostic, w.min_overlap, w.cache_slots,
-                    w.steps if steps is None else steps, w.append)
+                    w.steps if steps is None else steps, w.append, w.sink_blocks, w.window_blocks)
 
 
 def run_unit(cfg: OrcCfg, K: np.ndarray, V: np.ndarray, a: np.ndarray, q: np.ndarray,

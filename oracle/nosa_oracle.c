@@ -168,24 +168,28 @@ int orc_evict_update(const float* a, const int* ge_prev, int n_ge_prev, int n_fr
 /* a3: query-aware selection under the minimum-overlap constraint [S31][SE].   */
 /* ------------------------------------------------------------------------ */
 
-/* S(t) = Gamma_e(t) ∪ Gamma_q(t), with Gamma_q(t) drawn from blocks outside
- * Gamma_e(t) (the budget is divided between the two subsets).
+/* S(t) = F(t) ∪ Gamma_e(t) ∪ Gamma_q(t).  F(t) is the set of forced blocks
+ * (attention sink and sliding window, see orc_forced; empty unless
+ * configured).  Gamma_q(t) is drawn from blocks outside F(t) ∪ Gamma_e(t)
+ * (the budget is divided between the subsets).
  * Reading (gamma0): at most c_max = k - m blocks of S(t) may be absent from
- * S(t-1).  Blocks that Gamma_e(t) adds outside S(t-1) use that allowance first:
- *   c_t = max(0, c_max - |Gamma_e(t) \ S(t-1)|)
- *   O   = S(t-1) \ Gamma_e(t)                       (old candidates)
- *   N   = blocks outside Gamma_e(t) ∪ S(t-1)        (new candidates)
+ * S(t-1).  Forced and query-agnostic blocks that are new use that allowance
+ * first:
+ *   c_t = max(0, c_max - |(F(t) ∪ Gamma_e(t)) \ S(t-1)|)
+ *   O   = S(t-1) \ (F(t) ∪ Gamma_e(t))             (old candidates)
+ *   N   = blocks outside F(t) ∪ Gamma_e(t) ∪ S(t-1)  (new candidates)
  *   Gamma_q(t) = top-k_q of ( O ∪ top-c_t(N) )      by (score desc, id asc)
  * At the first step S(-1) is empty and there is no cap: Gamma_q(0) is the
- * top-k_q of every block outside Gamma_e(0).
- * sel_out gets S(t) ascending; returns |S(t)|. */
-int orc_select(const double* score, int n, const int* ge, int n_ge, const int* prev,
-               int n_prev, int first, int k_q, int c_max, int* sel_out) {
-  unsigned char* in_e = (unsigned char*)calloc((size_t)n + 1, 1);
+ * top-k_q of every block outside F(0) ∪ Gamma_e(0).
+ * forced: n flags (NULL = none).  sel_out gets S(t) ascending; returns |S(t)|. */
+int orc_select_forced(const double* score, int n, const unsigned char* forced, const int* ge, int n_ge,
+                      const int* prev, int n_prev, int first, int k_q, int c_max, int* sel_out) {
+  unsigned char* in_e = (unsigned char*)calloc((size_t)n + 1, 1);  /* F ∪ Gamma_e */
   unsigned char* in_p = (unsigned char*)calloc((size_t)n + 1, 1);
   orc_item* cand = (orc_item*)malloc(sizeof(orc_item) * (size_t)(n + 1));
   orc_item* newc = (orc_item*)malloc(sizeof(orc_item) * (size_t)(n + 1));
   for (int i = 0; i < n_ge; ++i) in_e[ge[i]] = 1;
+  if (forced) for (int j = 0; j < n; ++j) if (forced[j]) in_e[j] = 1;
   for (int i = 0; i < n_prev; ++i) if (prev[i] < n) in_p[prev[i]] = 1;
 
   int nc = 0;
@@ -194,7 +198,7 @@ int orc_select(const double* score, int n, const int* ge, int n_ge, const int* p
       if (!in_e[j]) { cand[nc].key = score[j]; cand[nc].idx = j; ++nc; }
   } else {
     int e_new = 0;
-    for (int i = 0; i < n_ge; ++i) if (!in_p[ge[i]]) ++e_new;
+    for (int j = 0; j < n; ++j) if (in_e[j] && !in_p[j]) ++e_new;
     int c_t = c_max - e_new;
     if (c_t < 0) c_t = 0;
     int nn = 0;
@@ -210,11 +214,32 @@ int orc_select(const double* score, int n, const int* ge, int n_ge, const int* p
   int nq = nc < k_q ? nc : k_q;
 
   int ns = 0;
-  for (int i = 0; i < n_ge; ++i) sel_out[ns++] = ge[i];
+  for (int j = 0; j < n; ++j) if (in_e[j]) sel_out[ns++] = j;
   for (int i = 0; i < nq; ++i) sel_out[ns++] = cand[i].idx;
   qsort(sel_out, (size_t)ns, sizeof(int), orc_int_cmp);
   free(in_e); free(in_p); free(cand); free(newc);
   return ns;
+}
+
+/* The selection without forced blocks. */
+int orc_select(const double* score, int n, const int* ge, int n_ge, const int* prev,
+               int n_prev, int first, int k_q, int c_max, int* sel_out) {
+  return orc_select_forced(score, n, NULL, ge, n_ge, prev, n_prev, first, k_q, c_max, sel_out);
+}
+
+/* Forced blocks (NOSA: Native and Offloadable Sparse Attention, paperlayer
+ * summary, App. B.2.2: one attention-sink block and 16 sliding-window blocks,
+ * counted inside the 48 query-agnostic blocks of NOSA's budget, and the same
+ * sink and window for InfLLMv2).  Reading: the sink is the first `sink`
+ * closed blocks, the window the last `window` closed blocks.  Flags n entries;
+ * returns how many are forced. */
+int orc_forced(int n, int sink, int window, unsigned char* is_forced) {
+  int c = 0;
+  for (int j = 0; j < n; ++j) {
+    is_forced[j] = (unsigned char)(j < sink || j >= n - window);
+    c += is_forced[j];
+  }
+  return c;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -319,6 +344,7 @@ typedef struct {
   int C;                 /* cache slots; 0 = KV resident on the GPU */
   int steps;
   int append;            /* 1: one token appended per step */
+  int sink, window;      /* forced blocks, counted inside k_e (0, 0 = none) */
 } orc_cfg;
 
 /* Per step t, in this order:
@@ -343,7 +369,9 @@ int orc_run_unit(const orc_cfg* cfg, const uint16_t* K, const uint16_t* V, const
                  int* out_resident, double* out_o, int* out_overlap, double* out_scores) {
   const int G = cfg->G, d = cfg->d, P = cfg->P, Q = cfg->Q, R = P / Q;
   const int k = cfg->k_q + cfg->k_e, c_max = k - cfg->m, C = cfg->C;
+  const int k_e_dyn = cfg->k_e - cfg->sink - cfg->window;  /* agnostic blocks beyond the forced ones */
   if (P % Q != 0 || k <= 0 || cfg->m > k || cfg->n0 > cfg->max_blocks) return -1;
+  if (k_e_dyn < 0 || cfg->sink < 0 || cfg->window < 0) return -1;
   if (C > 0 && C < k) return -2;
 
   uint16_t* kbar = (uint16_t*)calloc((size_t)cfg->max_blocks * R * d, sizeof(uint16_t));
@@ -357,6 +385,7 @@ int orc_run_unit(const orc_cfg* cfg, const uint16_t* K, const uint16_t* V, const
   int* fetch = (int*)malloc(sizeof(int) * (size_t)(k + 1));
   int* fetch_slot = (int*)malloc(sizeof(int) * (size_t)(k + 1));
   int* rows = (int*)malloc(sizeof(int) * (size_t)(k * P + P + 1));
+  unsigned char* forced = (unsigned char*)calloc((size_t)cfg->max_blocks + 1, 1);
   for (int c = 0; c < C; ++c) { slot_block[c] = -1; last_used[c] = -1; }
 
   int n = cfg->n0, tail = cfg->tail0, n_ge = 0, n_prev = 0, n_at_last_select = 0, rc = 0;
@@ -373,12 +402,19 @@ int orc_run_unit(const orc_cfg* cfg, const uint16_t* K, const uint16_t* V, const
         out_scores[(size_t)t * cfg->max_blocks + j] = j < n ? score[j] : NAN;
     }
     int first = (t == 0);
-    int n_e = orc_evict_update(a, ge, first ? 0 : n_ge, first ? 0 : n_at_last_select, n,
-                               cfg->k_e, ge_new);
+    /* Eligible for Gamma_e: closed blocks outside the sink and the window,
+     * [sink, n - window).  Blocks that became eligible since the last step
+     * (closed there, or slid out of the window) join its pool. */
+    orc_forced(n, cfg->sink, cfg->window, forced);
+    int e_to = n - cfg->window;
+    int e_from = first ? cfg->sink : n_at_last_select - cfg->window;
+    if (e_from < cfg->sink) e_from = cfg->sink;
+    if (e_to < e_from) e_to = e_from;
+    int n_e = orc_evict_update(a, ge, first ? 0 : n_ge, e_from, e_to, k_e_dyn, ge_new);
     memcpy(ge, ge_new, sizeof(int) * (size_t)n_e);
     n_ge = n_e;
     n_at_last_select = n;
-    int ns = orc_select(score, n, ge, n_ge, prev, n_prev, first, cfg->k_q, c_max, sel);
+    int ns = orc_select_forced(score, n, forced, ge, n_ge, prev, n_prev, first, cfg->k_q, c_max, sel);
 
     int ov = 0;
     for (int i = 0; i < ns; ++i)
@@ -423,7 +459,7 @@ int orc_run_unit(const orc_cfg* cfg, const uint16_t* K, const uint16_t* V, const
   }
 
   free(kbar); free(score); free(ge); free(ge_new); free(prev); free(sel);
-  free(slot_block); free(last_used); free(fetch); free(fetch_slot); free(rows);
+  free(slot_block); free(last_used); free(fetch); free(fetch_slot); free(rows); free(forced);
   return rc;
 }
 

@@ -498,3 +498,127 @@ def test_paper_budget_fixture(orc):
         ov = len(set(r["sel"].tolist()) & set(r["prev"]))
         assert ov >= k_e
         assert ov / k >= g["locality_lower_bound"]
+
+
+# --------------------------------------------------------------- forced blocks (sink, window)
+
+def brute_select_forced(score, n, F, E, prev, first, k_q, c_max):
+    F, E, prev = set(F), set(E), set(prev)
+    fixed = F | E
+    avail = [j for j in range(n) if j not in fixed]
+    new = set(j for j in avail if j not in prev)
+    c_t = 10 ** 9 if first else max(0, c_max - len(fixed - prev))
+    for r in range(min(k_q, len(avail)), -1, -1):
+        best, best_set = None, None
+        for comb in itertools.combinations(avail, r):
+            if not first and len(new.intersection(comb)) > c_t:
+                continue
+            val = sum(score[j] for j in comb)
+            if best is None or val > best:
+                best, best_set = val, comb
+        if best_set is not None:
+            return sorted(fixed | set(best_set))
+    return sorted(fixed)
+
+
+def test_forced_blocks_definition(orc):
+    assert orc.forced_blocks(10, 1, 3).tolist() == [0, 7, 8, 9]
+    assert orc.forced_blocks(10, 0, 0).tolist() == []
+    assert orc.forced_blocks(3, 1, 4).tolist() == [0, 1, 2]   # sink and window overlap
+
+
+def test_select_with_forced_blocks_equals_brute_force(orc):
+    rng = np.random.default_rng(16)
+    cases = 0
+    while cases < 200:
+        n = int(rng.integers(8, 13))
+        sink, window = int(rng.integers(0, 2)), int(rng.integers(0, 3))
+        F = orc.forced_blocks(n, sink, window).tolist()
+        k_e_dyn = int(rng.integers(0, 3))
+        k_q = int(rng.integers(1, 4))
+        free = [j for j in range(n) if j not in F]
+        if len(free) < k_e_dyn + k_q:
+            continue
+        E = sorted(rng.choice(free, size=k_e_dyn, replace=False).tolist())
+        k = len(F) + k_e_dyn + k_q
+        c_max = int(rng.integers(0, k + 1))
+        first = bool(rng.random() < 0.2)
+        prev = [] if first else sorted(rng.choice(n, size=min(k, n), replace=False).tolist())
+        score = rng.standard_normal(n)
+        got = orc.select_forced(score, F, E, prev, first, k_q, c_max)
+        assert got.tolist() == brute_select_forced(score, n, F, E, prev, first, k_q, c_max)
+        cases += 1
+
+
+def _run_policy(orc, n0, steps, k_q, k_e, m, sink, window, append, seed):
+    rng = np.random.default_rng(seed)
+    G, d, P = 2, 128, 64
+    max_blocks = n0 + (steps + P - 1) // P + 1 if append else n0
+    K = _rand_bf16(rng, (max_blocks * P, d))
+    V = _rand_bf16(rng, (max_blocks * P, d))
+    a = rng.random(max_blocks).astype(np.float32)
+    q = _rand_bf16(rng, (steps, G, d))
+    cfg = orc.make_cfg(G, d, P, 16, n0, 0, max_blocks, k_q, k_e, m, 0, steps, append, sink, window)
+    return orc.run_unit(cfg, K, V, a, q, attend_steps=[], want_scores=True), max_blocks
+
+
+def test_sliding_window_invariants_with_closing_blocks(orc):
+    """The sink and the last `window` closed blocks are in every S(t); the
+    window slides as blocks close; |S| = k; overlap >= m whenever the new
+    forced and agnostic blocks fit in the allowance."""
+    n0, steps, sink, window, k_q, k_e, m = 40, 300, 1, 6, 8, 12, 16
+    r, _ = _run_policy(orc, n0, steps, k_q, k_e, m, sink, window, True, 17)
+    k = k_q + k_e
+    for t in range(steps):
+        n = n0 + t // 64  # blocks closed before step t's selection
+        S = set(r.sel[t].tolist())
+        assert len(S) == k
+        assert set(orc.forced_blocks(n, sink, window).tolist()) <= S
+        if t > 0:
+            assert r.overlap[t] >= min(m, k - 2)
+
+
+def test_infllmv2_policy_is_forced_plus_plain_topk(orc):
+    """Sink + window + the query-aware top-k of the rest, with no agnostic set
+    and no overlap floor, is what InfLLMv2 selects (paperlayer summary,
+    App. B.2.2: 1 sink block, 16 window blocks, 47 dynamic blocks)."""
+    n0, steps = 200, 12
+    r, _ = _run_policy(orc, n0, steps, 47, 17, 0, 1, 16, False, 18)
+    F = set(orc.forced_blocks(n0, 1, 16).tolist())
+    for t in range(steps):
+        s = r.scores[t][:n0]
+        rest = np.array([j for j in range(n0) if j not in F])
+        top = rest[np.argsort(-s[rest], kind="stable")[:47]]
+        assert r.sel[t].tolist() == sorted(F | set(top.tolist()))
+
+
+def test_paper_split_with_sink_and_window_keeps_75_percent(orc):
+    """NOSA's own budget (App. B.2.2): 16 query-aware + 48 agnostic blocks, the
+    48 counting one sink and 16 window blocks; App. E: consecutive selections
+    share at least k_e = 48 of the 64 blocks."""
+    g = json.load(open(os.path.join(HERE, "golden", "paper_budget.json")))
+    r, _ = _run_policy(orc, 256, 40, g["query_aware_blocks"], g["agnostic_blocks"], 0,
+                       g["infllmv2_sink_blocks"], g["infllmv2_window_blocks"], False, 19)
+    for t in range(1, 40):
+        assert r.overlap[t] >= g["agnostic_blocks"]
+        assert r.overlap[t] / 64 >= g["locality_lower_bound"]
+
+
+def test_block_leaving_the_window_joins_the_agnostic_pool(orc):
+    """A block that slides out of the window becomes eligible for Gamma_e; with
+    the highest agnostic score it is selected at every later step."""
+    rng = np.random.default_rng(20)
+    G, d, P, n0, steps = 2, 128, 64, 10, 190
+    max_blocks = 14
+    K = _rand_bf16(rng, (max_blocks * P, d))
+    V = _rand_bf16(rng, (max_blocks * P, d))
+    a = np.full(max_blocks, 0.1, dtype=np.float32)
+    a[10] = 2.0  # block 10 closes at step 63 and leaves the 1-block window at step 128
+    q = _rand_bf16(rng, (steps, G, d))
+    cfg = orc.make_cfg(G, d, P, 16, n0, 0, max_blocks, 3, 2, 0, 0, steps, True, 0, 1)
+    r = orc.run_unit(cfg, K, V, a, q, attend_steps=[])
+    for t in range(64, 128):
+        assert 10 in r.sel[t].tolist()          # in the window
+    for t in range(128, steps):
+        assert 10 in r.sel[t].tolist()          # now through Gamma_e
+        assert 11 in r.sel[t].tolist()          # the new window block
