@@ -46,6 +46,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=8)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="offload_b64")
+    p.add_argument("--policy", default="nosa", choices=["nosa", "paper", "infllmv2", "full"],
+                   help="selection policy on the same kernels (see configs.POLICIES)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=50)
     return p.parse_args()
@@ -260,7 +262,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     build.build()
 
-    base = configs.get(args.workload)
+    base = configs.with_policy(configs.get(args.workload), args.policy)
     total = 1 + args.warmup + 1 + args.steps + 2 * min(args.steps, 50) + args.e2e_steps + 8
     w = base.with_(steps=max(base.steps, total))
     data = inputs.generate(w)
@@ -356,11 +358,12 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 K/V, U(0,1) agnostic scores, AR(1) queries)",
-            "config": {"workload": w.name, "batch": w.batch, "context": w.context,
+            "config": {"workload": w.name, "policy": args.policy, "batch": w.batch, "context": w.context,
                        "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                        "block": w.block, "sub_block": w.sub_block, "k": w.k, "k_query": w.k_query,
-                       "k_agnostic": w.k_agnostic, "min_overlap": w.min_overlap,
-                       "cache_slots": w.cache_slots, "kv": "pinned host", "parallelism": f"replicas x{world}",
+                       "k_agnostic": w.k_agnostic, "min_overlap": w.min_overlap, "sink_blocks": w.sink_blocks,
+                       "window_blocks": w.window_blocks, "cache_slots": w.cache_slots,
+                       "kv": "pinned host" if w.offloaded else "HBM", "parallelism": f"replicas x{world}",
                        "l2": "per-step traffic 288 MiB > 126 MB L2, no flush", "graph": "cuda graph replay"},
             "roofline": dominant,
             "roofline_other": other,

@@ -88,6 +88,10 @@ typedef struct {
   int max_blocks;     /* block capacity per unit (prompt + growth), >= k, <= 8192 */
   int cache_slots;    /* 0: KV resident in HBM; else GPU cache blocks per unit,
                          k <= cache_slots <= 1024, KV in pinned host memory */
+  int sink_blocks;    /* forced: the first sink_blocks closed blocks (attention sink) */
+  int window_blocks;  /* forced: the last window_blocks closed blocks (sliding window);
+                         sink + window <= k_agnostic: forced blocks count inside the
+                         query-agnostic budget (NOSA summary App. B.2.2) */
 } nosa_config;
 
 /* Running totals since the last attach or nosa_reset_stats. */
@@ -151,14 +155,16 @@ NOSA_API nosa_status nosa_append_token(nosa_ctx* ctx, const void* k_new, const v
  * scores: device fp64 [U, max_blocks]; entries j >= n are left untouched. */
 NOSA_API nosa_status nosa_score_blocks(nosa_ctx* ctx, const void* q, double* scores, nosa_stream_t stream);
 
-/* Selection (NOSA summary §2.1, §3.1, App. E), per unit:
- *   Gamma_e(t) = top-k_e by agnostic score of Gamma_e(t-1) plus the blocks
- *                closed since the last step (all closed blocks at step 0);
- *                an evicted block never re-enters Gamma_e.
- *   c_t        = max(0, (k - m) - |Gamma_e(t) \ S(t-1)|)   (no cap at step 0)
- *   Gamma_q(t) = top-k_q by score of (S(t-1) \ Gamma_e(t)) ∪ top-c_t of the
- *                blocks in neither Gamma_e(t) nor S(t-1)
- *   S(t)       = Gamma_e(t) ∪ Gamma_q(t)
+/* Selection (NOSA summary §2.1, §3.1, App. B.2.2, App. E), per unit, with
+ * F(t) the forced blocks (first sink_blocks and last window_blocks closed):
+ *   Gamma_e(t) = top-(k_e - |F|) by agnostic score of Gamma_e(t-1) plus the
+ *                blocks that became eligible (closed outside the window, or
+ *                slid out of it) since the last step (all eligible blocks at
+ *                step 0); an evicted block never re-enters Gamma_e.
+ *   c_t        = max(0, (k - m) - |(F ∪ Gamma_e)(t) \ S(t-1)|)   (no cap at step 0)
+ *   Gamma_q(t) = top-k_q by score of (S(t-1) \ (F ∪ Gamma_e)(t)) ∪ top-c_t of
+ *                the blocks in neither (F ∪ Gamma_e)(t) nor S(t-1)
+ *   S(t)       = F(t) ∪ Gamma_e(t) ∪ Gamma_q(t)
  * Ties go to the lower block id.  scores: device fp64 as written by
  * nosa_score_blocks.  sel: device int32 [U, k], S(t) ascending, -1 padded. */
 NOSA_API nosa_status nosa_select(nosa_ctx* ctx, const double* scores, int32_t* sel, nosa_stream_t stream);

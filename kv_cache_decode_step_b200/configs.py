@@ -138,3 +138,32 @@ def describe(w: Workload) -> str:
             f"n={w.n_blocks0} k={w.k}({w.k_query}+{w.k_agnostic}) m={w.min_overlap} "
             f"steps={w.steps} {mode}" + (f" C={w.cache_slots}" if w.offloaded else "")
             + (" append" if w.append else ""))
+
+
+# Selection policies on the same kernels (NOSA: Native and Offloadable Sparse
+# Attention, paperlayer summary, App. B.2.2, for a 64-block = 4096-token budget):
+#   nosa     -- the workload's own split and overlap floor
+#   paper    -- NOSA's own split: 16 query-aware + 48 agnostic blocks, the 48
+#               counting one sink block and 16 sliding-window blocks, no floor
+#               beyond what the split guarantees (App. E: 48 of 64)
+#   infllmv2 -- 1 sink + 16 window + 47 query-aware blocks, no agnostic set,
+#               no overlap floor
+#   full     -- every closed block, KV resident (dense attention)
+POLICIES = ("nosa", "paper", "infllmv2", "full")
+
+
+def with_policy(w: Workload, policy: str) -> Workload:
+    if policy == "nosa":
+        return w
+    if policy == "paper":
+        return w.with_(name=f"{w.name}/paper", k_query=16, k_agnostic=48, sink_blocks=1, window_blocks=16,
+                       min_overlap=0, gamma0=0.0)
+    if policy == "infllmv2":
+        return w.with_(name=f"{w.name}/infllmv2", k_query=47, k_agnostic=17, sink_blocks=1, window_blocks=16,
+                       min_overlap=0, gamma0=0.0)
+    if policy == "full":
+        if w.append:
+            raise ValueError("the dense policy covers fixed-length workloads")
+        return w.with_(name=f"{w.name}/full", k_query=w.n_blocks0, k_agnostic=0, min_overlap=0, gamma0=0.0,
+                       offloaded=False, cache_factor=0)
+    raise ValueError(f"unknown policy {policy!r}")

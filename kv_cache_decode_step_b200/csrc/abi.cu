@@ -149,6 +149,9 @@ nosa_status validate(const nosa_config* c) {
     return fail(NOSA_ERR_INVALID, "min_overlap %d outside [0, k=%d]", c->min_overlap, k);
   if (c->max_blocks < k || c->max_blocks > 8192)
     return fail(NOSA_ERR_INVALID, "max_blocks %d outside [k=%d, 8192]", c->max_blocks, k);
+  if (c->sink_blocks < 0 || c->window_blocks < 0 || c->sink_blocks + c->window_blocks > c->k_agnostic)
+    return fail(NOSA_ERR_INVALID, "need sink_blocks, window_blocks >= 0 and sink + window <= k_agnostic (%d)",
+                c->k_agnostic);
   if (c->cache_slots != 0 && (c->cache_slots < k || c->cache_slots > 1024))
     return fail(NOSA_ERR_INVALID, "cache_slots %d must be 0 or in [k=%d, 1024]", c->cache_slots, k);
   const long long U = (long long)c->batch * c->n_kv_heads;
@@ -465,6 +468,8 @@ nosa_status nosa_select(nosa_ctx* c, const double* scores, int32_t* sel, nosa_st
   a.k = c->k;
   a.c_max = c->k - c->cfg.min_overlap;
   a.words = c->words;
+  a.sink = c->cfg.sink_blocks;
+  a.window = c->cfg.window_blocks;
   NOSA_CUDA(launch_select(a, reinterpret_cast<cudaStream_t>(stream)));
   c->phase = kSelected;
   return NOSA_OK;

@@ -224,6 +224,7 @@ struct SelectArgs {
   DevState* ds;
   DevStats* st;
   int U, max_blocks, k_q, k_e, k, c_max, words;
+  int sink, window;         // forced blocks, counted inside k_e
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 

@@ -9,11 +9,14 @@
 // NOSA (gist.science explainer), technical summary, Method: a block dropped by
 // the query-agnostic part is never taken back by it.
 //
-// Per unit and step t (S(-1) empty):
-//   Gamma_e(t) = top-k_e by agnostic score of Gamma_e(t-1) ∪ {newly closed}
-//   c_t        = max(0, (k - m) - |Gamma_e(t) \ S(t-1)|), unbounded at t = 0
-//   Gamma_q(t) = top-k_q by score of (S(t-1) \ Gamma_e(t)) ∪ top-c_t(new)
-//   S(t)       = Gamma_e(t) ∪ Gamma_q(t), ties to the lower block id.
+// Per unit and step t (S(-1) empty), F(t) = forced blocks (the first `sink`
+// and last `window` closed blocks; App. B.2.2 counts them inside NOSA's
+// query-agnostic budget):
+//   Gamma_e(t) = top-(k_e - |F|) by agnostic score of Gamma_e(t-1) ∪ {blocks
+//                that became eligible: closed outside the window or slid out}
+//   c_t        = max(0, (k - m) - |(F ∪ Gamma_e)(t) \ S(t-1)|), unbounded at t = 0
+//   Gamma_q(t) = top-k_q by score of (S(t-1) \ (F ∪ Gamma_e)) ∪ top-c_t(new)
+//   S(t)       = F(t) ∪ Gamma_e(t) ∪ Gamma_q(t), ties to the lower block id.
 //
 // Lane l owns the blocks j with j % 32 == l.  Up to 1024 blocks their keys sit
 // in registers and sets are per-lane bit masks; beyond that sets are bitmaps
@@ -212,15 +215,23 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectArgs a) {
   }
   __syncwarp();
 
-  // ---- Gamma_e: unchanged unless this is the first step or blocks closed
+  // ---- Gamma_e over the eligible blocks [sink, n - window): unchanged
+  // unless this is the first step or blocks became eligible since the last
   const Keys KA{nullptr, ag, nullptr, false};
   const Keys KS{stage ? skeys : nullptr, nullptr, sc, false};
-  if (first || n_from < n) {
-    const int pool_lo = first ? 0 : n_from;
-    for (int w = lane; w < nw; w += 32) bmE[w] |= valid_bits(w, n) & ~valid_bits(w, pool_lo);
+  const int e_to = n - a.window;
+  const int e_from = max(a.sink, first ? a.sink : n_from - a.window);
+  if (e_from < e_to) {
+    for (int w = lane; w < nw; w += 32) bmE[w] |= valid_bits(w, e_to) & ~valid_bits(w, e_from);
     __syncwarp();
-    keep_best(bmE, bmT, nw, a.k_e, lane, KA);
+    keep_best(bmE, bmT, nw, a.k_e - a.sink - a.window, lane, KA);
   }
+  const int ne = bitmap_to_list(bmE, nw, ge, a.k_e, lane);
+  for (int i = ne + lane; i < a.k_e; i += 32) ge[i] = -1;
+  // from here on bmE holds F(t) ∪ Gamma_e(t): the sink and the window join it
+  for (int w = lane; w < nw; w += 32)
+    bmE[w] |= valid_bits(w, min(a.sink, n)) | (valid_bits(w, n) & ~valid_bits(w, max(0, n - a.window)));
+  __syncwarp();
 
   // ---- Gamma_q
   if (first) {
@@ -257,8 +268,6 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(SelectArgs a) {
     if (i >= ns) sel[i] = -1;
     prev[i] = v;
   }
-  const int ne = bitmap_to_list(bmE, nw, ge, a.k_e, lane);
-  for (int i = ne + lane; i < a.k_e; i += 32) ge[i] = -1;
 
   if (lane == 0) {
     atomicAdd(&a.st->selected, (unsigned long long)ns);
@@ -365,14 +374,18 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_reg_kernel(SelectArgs a
   int* ge = a.ge + (size_t)u * a.k_e;
 
   unsigned long long ks[R];
-  uint32_t valid = 0u, fresh = 0u;  // closed blocks; blocks closed since the last step
-  const int pool_lo = first ? 0 : n_from;
+  // closed blocks; blocks that became eligible for Gamma_e since the last
+  // step ([sink, n - window) minus what was eligible then); forced blocks
+  uint32_t valid = 0u, fresh = 0u, forced = 0u;
+  const int e_to = n - a.window;
+  const int e_from = max(a.sink, first ? a.sink : n_from - a.window);
 #pragma unroll
   for (int i = 0; i < R; ++i) {
     const int j = 32 * i + lane;
     ks[i] = j < n ? key_f64(sc[j]) : 0ull;
     if (j < n) valid |= 1u << i;
-    if (j < n && j >= pool_lo) fresh |= 1u << i;
+    if (j >= e_from && j < e_to) fresh |= 1u << i;
+    if (j < n && (j < a.sink || j >= n - a.window)) forced |= 1u << i;
   }
   for (int i = lane; i < 2 * R; i += 32) (&sbm[warp][0][0])[i] = 0u;
   __syncwarp();
@@ -394,7 +407,8 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_reg_kernel(SelectArgs a
     mE |= ((sbm[warp][1][i] >> lane) & 1u) << i;
   }
 
-  // ---- Gamma_e: unchanged unless this is the first step or blocks closed
+  // ---- Gamma_e over the eligible blocks: unchanged unless this is the first
+  // step or blocks became eligible since the last
   if (__any_sync(kFull, fresh != 0u)) {
     unsigned long long ka[R];
 #pragma unroll
@@ -403,22 +417,23 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_reg_kernel(SelectArgs a
       ka[i] = j < n ? key_f32(ag[j]) : 0ull;
     }
     mE |= fresh;
-    keep_best_reg<R>(mE, a.k_e, ka, lane);
+    keep_best_reg<R>(mE, a.k_e - a.sink - a.window, ka, lane);
   }
 
-  // ---- Gamma_q
+  // ---- Gamma_q, outside F(t) ∪ Gamma_e(t)
+  const uint32_t mF = mE | forced;
   uint32_t mX;
   if (first) {
-    mX = valid & ~mE;
+    mX = valid & ~mF;
   } else {
-    const int e_new = (int)__reduce_add_sync(kFull, (unsigned)__popc(mE & ~mP));
+    const int e_new = (int)__reduce_add_sync(kFull, (unsigned)__popc(mF & ~mP));
     const int c_t = max(0, a.c_max - e_new);
-    mX = valid & ~mE & ~mP;  // new candidates
+    mX = valid & ~mF & ~mP;  // new candidates
     keep_best_reg<R>(mX, c_t, ks, lane);
-    mX |= mP & ~mE;          // ∪ old candidates
+    mX |= mP & ~mF;          // ∪ old candidates
   }
   keep_best_reg<R>(mX, a.k_q, ks, lane);
-  const uint32_t mS = mX | mE;
+  const uint32_t mS = mX | mF;
   const int ov = (int)__reduce_add_sync(kFull, (unsigned)__popc(mS & mP));
 
   int* sel = a.sel + (size_t)u * a.k;

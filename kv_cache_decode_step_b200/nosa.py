@@ -43,7 +43,7 @@ class NosaError(RuntimeError):
 class nosa_config(C.Structure):
     _fields_ = [(n, C.c_int) for n in (
         "batch", "n_q_heads", "n_kv_heads", "head_dim", "block", "sub_block", "k_query",
-        "k_agnostic", "min_overlap", "max_blocks", "cache_slots")]
+        "k_agnostic", "min_overlap", "max_blocks", "cache_slots", "sink_blocks", "window_blocks")]
 
 
 class nosa_stats(C.Structure):
@@ -221,4 +221,5 @@ def nosa_sparse_decode_noalloc(q, k, v, batch: int, n_q_heads: int, n_kv_heads: 
 
 def config_from_workload(w) -> nosa_config:
     return nosa_config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.sub_block,
-                       w.k_query, w.k_agnostic, w.min_overlap, w.max_blocks, w.cache_slots)
+                       w.k_query, w.k_agnostic, w.min_overlap, w.max_blocks, w.cache_slots,
+                       w.sink_blocks, w.window_blocks)

@@ -63,6 +63,8 @@ def _cfg(**kw):
     ("max_blocks", 9000, nosa.NOSA_ERR_INVALID),
     ("cache_slots", 15, nosa.NOSA_ERR_INVALID),       # 0 < C < k
     ("cache_slots", 2000, nosa.NOSA_ERR_INVALID),
+    ("sink_blocks", -1, nosa.NOSA_ERR_INVALID),
+    ("window_blocks", 5, nosa.NOSA_ERR_INVALID),     # sink + window > k_agnostic = 4
 ])
 def test_create_rejects_bad_configs(L, field, value, status):
     out = C.c_void_p()
