@@ -48,6 +48,8 @@ def parse():
     p.add_argument("--workload", default="offload_b64")
     p.add_argument("--policy", default="nosa", choices=["nosa", "paper", "infllmv2", "full"],
                    help="selection policy on the same kernels (see configs.POLICIES)")
+    p.add_argument("--k-query", type=int, default=None,
+                   help="query-aware blocks of the 64-block budget (paper policy; default 16)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=50)
     return p.parse_args()
@@ -262,7 +264,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     build.build()
 
-    base = configs.with_policy(configs.get(args.workload), args.policy)
+    base = configs.with_policy(configs.get(args.workload), args.policy, args.k_query)
     total = 1 + args.warmup + 1 + args.steps + 2 * min(args.steps, 50) + args.e2e_steps + 8
     w = base.with_(steps=max(base.steps, total))
     data = inputs.generate(w)

@@ -152,12 +152,17 @@ def describe(w: Workload) -> str:
 POLICIES = ("nosa", "paper", "infllmv2", "full")
 
 
-def with_policy(w: Workload, policy: str) -> Workload:
+def with_policy(w: Workload, policy: str, k_query: Optional[int] = None) -> Workload:
+    """k_query (paper policy only) moves the query-aware share of the 64-block
+    budget; the rest stays query-agnostic, sink and window included."""
     if policy == "nosa":
         return w
     if policy == "paper":
-        return w.with_(name=f"{w.name}/paper", k_query=16, k_agnostic=48, sink_blocks=1, window_blocks=16,
-                       min_overlap=0, gamma0=0.0)
+        kq = 16 if k_query is None else int(k_query)
+        if not 0 <= kq <= 64 - 17:
+            raise ValueError("the paper split keeps 1 sink + 16 window blocks: k_query in [0, 47]")
+        return w.with_(name=f"{w.name}/paper" + ("" if k_query is None else f"-kq{kq}"), k_query=kq,
+                       k_agnostic=64 - kq, sink_blocks=1, window_blocks=16, min_overlap=0, gamma0=0.0)
     if policy == "infllmv2":
         return w.with_(name=f"{w.name}/infllmv2", k_query=47, k_agnostic=17, sink_blocks=1, window_blocks=16,
                        min_overlap=0, gamma0=0.0)
