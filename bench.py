@@ -31,6 +31,8 @@ import subprocess
 import sys
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -265,7 +267,7 @@ def run_ours(args):
     build.build()
 
     base = configs.with_policy(configs.get(args.workload), args.policy, args.k_query)
-    total = 1 + args.warmup + 1 + args.steps + 2 * min(args.steps, 50) + 2 * args.e2e_steps + 8
+    total = 1 + args.warmup + 1 + args.steps + 2 * min(args.steps, 50) + 2 * args.e2e_steps + LATENCY_STEPS + 8
     w = base.with_(steps=max(base.steps, total))
     data = inputs.generate(w)
     dec = runner.Decoder(w, data, device=local)
@@ -328,14 +330,17 @@ def run_ours(args):
                      "side-stream pass, attention_ms (both attention launches + combine + advance) from a "
                      "single-stream pass where the gather has finished before attention starts")
 
+    latency = step_latency_pass(torch, dec, w, LATENCY_STEPS)
+
     # ---- end to end through host buffers: q from pinned host, out to pinned host
     e2e = e2e_pass(torch, dec, w, nosa, args.e2e_steps)
     e2e["eager_value"] = e2e_pass(torch, dec, w, nosa, args.e2e_steps, eager=True)["value"]
 
     # kernels per step: score, select, [plan, gather, misses pass], hits pass;
     # with appends also append, close and advance (otherwise the last
-    # attention CTA ends the step)
-    launches_per_step = (6 if w.offloaded else 3) + (3 if w.append else 0)
+    # attention CTA ends the step), and with KV in host memory the
+    # write-through of a block the previous step closed
+    launches_per_step = (6 if w.offloaded else 3) + (3 if w.append else 0) + (1 if w.append and w.offloaded else 0)
     gather_ms = phase["gather_ms"]
     attn_ms = phase["attention_ms"]
     gather_gbs = (phase["fetched_bytes_per_step"] / (gather_ms * 1e-3) / 1e9) if gather_ms > 0 else 0.0
@@ -387,6 +392,7 @@ def run_ours(args):
             },
             "phases_ms": phase,
             "e2e": e2e,
+            "step_latency_us": latency,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -447,6 +453,35 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
     out["fetched_bytes_per_step"] = (dec.stats()["fetched_bytes"] - fb0) / n
     out["steps"] = n
     out["single_stream"] = bool(single_stream)
+    return out
+
+
+LATENCY_STEPS = 256
+
+
+def step_latency_pass(torch, dec, w, n):
+    """Per-step device time of n graph replays queued back to back (an event
+    between consecutive steps).  With growing sequences, the steps whose
+    appended token fills the tail block (and so close it) are reported apart."""
+    s = dec.stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    steps = []
+    torch.cuda.synchronize()
+    for i in range(n):
+        steps.append(dec.t)
+        ev[i].record(s)
+        dec.replay()
+    ev[n].record(s)
+    torch.cuda.synchronize()
+    us = np.array([ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(n)])
+    out = {"n": n, "mean": float(us.mean()), "p50": float(np.percentile(us, 50)),
+           "p90": float(np.percentile(us, 90)), "p99": float(np.percentile(us, 99)), "max": float(us.max())}
+    if w.append:
+        close = np.array([(w.context + t + 1) % w.block == 0 for t in steps])
+        out["close_steps"] = int(close.sum())
+        out["close_mean"] = float(us[close].mean()) if close.any() else None
+        out["other_mean"] = float(us[~close].mean())
+        out["other_max"] = float(us[~close].max())
     return out
 
 

@@ -143,8 +143,16 @@ NOSA_API nosa_status nosa_attach_kv(nosa_ctx* ctx, const void* k, const void* v,
  * k_new, v_new: device bf16 [B, H_kv, d].  agnostic_if_close: device fp32 [U]
  * or NULL; it becomes the agnostic score of the tail block if this token fills
  * it, in which case nosa_sparse_decode closes the block at the end of the step
- * (pooled keys built, written through to the host KV, candidate from the next
- * step on).  NOSA_ERR_INVALID when the unit would exceed max_blocks*P tokens. */
+ * (pooled keys built, candidate from the next step on).  A closed block's K/V
+ * reach the attached KV at once when it is device memory.  When it is host
+ * memory they are staged in HBM and written through while the next step runs
+ * (a low-priority kernel on a stream of the context, forked by
+ * nosa_score_blocks and joined by nosa_sparse_decode); until then the miss
+ * gather reads the staged copy.  nosa_get_state, nosa_set_state and
+ * nosa_attach_kv land a pending write-through first, so after a step the host
+ * copy of the last closed block is complete once the next step has run or one
+ * of those calls has returned.
+ * NOSA_ERR_INVALID when the unit would exceed max_blocks*P tokens. */
 NOSA_API nosa_status nosa_append_token(nosa_ctx* ctx, const void* k_new, const void* v_new,
                               const float* agnostic_if_close, nosa_stream_t stream);
 
@@ -217,6 +225,26 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
                                                 int n_q_heads, int n_kv_heads, int max_blocks,
                                                 const int32_t* sel, int k_sel, void* out,
                                                 nosa_stream_t stream);
+
+/* Row gather at a chosen granularity (NOSA summary §3.2 and §4: block-wise
+ * transfer of 16 KiB blocks against element-wise transfer of single tokens).
+ * For i < n: row dst_idx[i] of dst  <-  row src_idx[i] of src, each row
+ * row_bytes long (a power of two in [16, 65536]); dst_idx = NULL means row i.
+ * A miss of the decode step is two 16 KiB rows (its K and its V block); a
+ * token is two 256-byte rows at d = 128, bf16.
+ * src: device-addressable memory of src_rows rows (pinned host memory mapped
+ * into the device's address space, or device memory); dst: device memory of
+ * dst_rows rows; both 16-byte aligned.  src_idx, dst_idx: device int64 [n].
+ * ctas: CTAs of 256 threads, 0 for a quarter of the SMs (the decode step's
+ * gather width).  flags: device uint32 or NULL; bit 0 is ORed in when an
+ * index is out of range, and that row is skipped.  Destination rows must be
+ * distinct (two copies into one row race).  Asynchronous on stream; n = 0
+ * launches nothing.  NOSA_ERR_INVALID for bad sizes, NULL pointers, a src the
+ * device cannot address (pageable host memory) or a dst, index or flags
+ * pointer that is not device memory. */
+NOSA_API nosa_status nosa_gather_rows(const void* src, int64_t src_rows, void* dst, int64_t dst_rows,
+                                      int32_t row_bytes, const int64_t* src_idx, const int64_t* dst_idx,
+                                      int32_t n, int32_t ctas, uint32_t* flags, nosa_stream_t stream);
 
 /* Synchronous.  Copies the running totals into *stats. */
 NOSA_API nosa_status nosa_get_stats(nosa_ctx* ctx, nosa_stats* stats);

@@ -50,6 +50,30 @@ enum Phase { kReady = 0, kScored = 1, kSelected = 2, kFetched = 3 };
 
 void nosa::record_error(const char* msg) { g_err = msg ? msg : ""; }
 
+// Classify a pointer: 1 device memory of this device, 2 pinned/registered
+// host memory (device-addressable), 0 other.
+int nosa::pointer_kind(const void* p, void** dev_ptr) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+    *dev_ptr = const_cast<void*>(p);
+    return 1;
+  }
+  if (at.type == cudaMemoryTypeHost) {
+    void* d = nullptr;
+    if (cudaHostGetDevicePointer(&d, const_cast<void*>(p), 0) != cudaSuccess || !d) {
+      cudaGetLastError();
+      return 0;
+    }
+    *dev_ptr = d;
+    return 2;
+  }
+  return 0;
+}
+
 struct nosa_ctx {
   nosa_config cfg{};
   int U = 0, G = 0, k = 0, C = 0, max_blocks = 0, words = 0, device = 0;
@@ -96,6 +120,16 @@ struct nosa_ctx {
   int nparts = 2, gather_grid = 148, attn_grid = 296;
   int* unit_done = nullptr;
   int* done_ctr = nullptr;
+
+  // overlapped write-through of closed blocks (KV in host memory): the close
+  // kernel stages a closed block in HBM; a low-priority kernel on wt_stream
+  // copies it to the host store during the next step
+  uint16_t* stage_k = nullptr;
+  uint16_t* stage_v = nullptr;
+  cudaStream_t wt_stream = nullptr;
+  cudaEvent_t ev_wt_fork = nullptr, ev_wt_done = nullptr;
+  bool wt_forked = false;
+  int wt_grid = 18;
 };
 
 namespace {
@@ -178,40 +212,42 @@ void free_all(nosa_ctx* c) {
   void* ptrs[] = {c->kbar,   c->agnostic,   c->ge,        c->prev,   c->cache_k,   c->cache_v,
                   c->slot_block, c->last_used, c->block_slot, c->items, c->n_hit,   c->n_items,
                   c->glist,  c->tail_k,     c->tail_v,    c->a_pending, c->part_o, c->part_ml,
-                  c->ds,     c->st,         c->refill_count, c->unit_done, c->done_ctr};
+                  c->ds,     c->st,         c->refill_count, c->unit_done, c->done_ctr, c->stage_k,
+                  c->stage_v};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (c->ev_plan) cudaEventDestroy(c->ev_plan);
   if (c->ev_gather) cudaEventDestroy(c->ev_gather);
+  if (c->ev_wt_fork) cudaEventDestroy(c->ev_wt_fork);
+  if (c->ev_wt_done) cudaEventDestroy(c->ev_wt_done);
+  if (c->wt_stream) cudaStreamDestroy(c->wt_stream);
+}
+
+WriteThroughArgs write_through_args(const nosa_ctx* c) {
+  WriteThroughArgs w{};
+  w.stage_k = c->stage_k;
+  w.stage_v = c->stage_v;
+  w.kv_k = c->kv_k;
+  w.kv_v = c->kv_v;
+  w.ds = c->ds;
+  w.U = c->U;
+  w.max_blocks = c->max_blocks;
+  return w;
+}
+
+// Synchronous: lands a staged block that has not been written through yet
+// (the last step closed a block) in the host store.
+nosa_status flush_write_through(nosa_ctx* c) {
+  if (!c->stage_k || !c->attached) return NOSA_OK;
+  NOSA_CUDA(cudaDeviceSynchronize());  // the close that staged the block may still run
+  NOSA_CUDA(launch_write_through(write_through_args(c), c->wt_grid, c->wt_stream));
+  NOSA_CUDA(cudaStreamSynchronize(c->wt_stream));
+  return NOSA_OK;
 }
 
 nosa_status set_device(nosa_ctx* c) {
   NOSA_CUDA(cudaSetDevice(c->device));
   return NOSA_OK;
-}
-
-// Classify a pointer: 1 device memory of this device, 2 pinned/registered
-// host memory (device-addressable), 0 other.
-int pointer_kind(const void* p, void** dev_ptr) {
-  cudaPointerAttributes at{};
-  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
-    *dev_ptr = const_cast<void*>(p);
-    return 1;
-  }
-  if (at.type == cudaMemoryTypeHost) {
-    void* d = nullptr;
-    if (cudaHostGetDevicePointer(&d, const_cast<void*>(p), 0) != cudaSuccess || !d) {
-      cudaGetLastError();
-      return 0;
-    }
-    *dev_ptr = d;
-    return 2;
-  }
-  return 0;
 }
 
 }  // namespace
@@ -293,6 +329,8 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
     ALLOC(c->last_used, U * CS);
     ALLOC(c->block_slot, U * MB);
     ALLOC(c->glist, U * (CS > K ? CS : K));
+    ALLOC(c->stage_k, U * kP * kD);
+    ALLOC(c->stage_v, U * kP * kD);
   }
 #undef ALLOC
   auto cleanup = [&](nosa_status st) {
@@ -310,6 +348,15 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   if (cudaEventCreateWithFlags(&c->ev_plan, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_gather, cudaEventDisableTiming) != cudaSuccess)
     return cleanup(fail(NOSA_ERR_CUDA, "cudaEventCreate failed"));
+  if (c->offloaded) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&c->wt_stream, cudaStreamNonBlocking, least) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->ev_wt_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->ev_wt_done, cudaEventDisableTiming) != cudaSuccess)
+      return cleanup(fail(NOSA_ERR_CUDA, "write-through stream setup failed"));
+    c->wt_grid = (sms + 7) / 8;
+  }
   if ((s = make_row_map(&c->maps.tk, c->tail_k, U * kP)) != NOSA_OK) return cleanup(s);
   if ((s = make_row_map(&c->maps.tv, c->tail_v, U * kP)) != NOSA_OK) return cleanup(s);
   if (c->offloaded) {
@@ -353,6 +400,8 @@ nosa_status nosa_attach_kv(nosa_ctx* c, const void* k, const void* v, int n_toke
                 c->max_blocks * kP);
   nosa_status s = set_device(c);
   if (s != NOSA_OK) return s;
+  // a block the previous attachment closed last still belongs in its store
+  if ((s = flush_write_through(c)) != NOSA_OK) return s;
   void *dk = nullptr, *dv = nullptr, *da = nullptr;
   const int kk = pointer_kind(k, &dk), kv = pointer_kind(v, &dv), ka = pointer_kind(agnostic, &da);
   if (c->offloaded) {
@@ -442,7 +491,17 @@ nosa_status nosa_score_blocks(nosa_ctx* c, const void* q, double* scores, nosa_s
   a.Hkv = c->cfg.n_kv_heads;
   a.G = c->G;
   a.max_blocks = c->max_blocks;
-  NOSA_CUDA(launch_score(a, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (c->stage_k && c->appends_enabled) {
+    // a block closed by the previous step goes to the host store while this
+    // step runs; nosa_sparse_decode joins it before the next close
+    NOSA_CUDA(cudaEventRecord(c->ev_wt_fork, st));
+    NOSA_CUDA(cudaStreamWaitEvent(c->wt_stream, c->ev_wt_fork, 0));
+    NOSA_CUDA(launch_write_through(write_through_args(c), c->wt_grid, c->wt_stream));
+    NOSA_CUDA(cudaEventRecord(c->ev_wt_done, c->wt_stream));
+    c->wt_forked = true;
+  }
+  NOSA_CUDA(launch_score(a, st));
   c->phase = kScored;
   return NOSA_OK;
 }
@@ -516,6 +575,8 @@ nosa_status nosa_fetch_missing(nosa_ctx* c, const int32_t* sel, int32_t* fetch, 
   g.cv = c->cache_v;
   g.glist = c->glist;
   g.count = &c->ds->gather_count;
+  g.stage_k = c->stage_k;
+  g.stage_v = c->stage_v;
   g.ds = c->ds;
   g.U = c->U;
   g.C = c->C;
@@ -590,9 +651,15 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
     cl.agnostic = c->agnostic;
     cl.kv_k = c->kv_k;
     cl.kv_v = c->kv_v;
+    cl.stage_k = c->stage_k;
+    cl.stage_v = c->stage_v;
     cl.ds = c->ds;
     cl.U = c->U;
     cl.max_blocks = c->max_blocks;
+    if (c->wt_forked) {
+      NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_wt_done, 0));
+      c->wt_forked = false;
+    }
     NOSA_CUDA(launch_close(cl, st));
   }
   if (!fold_advance) NOSA_CUDA(launch_advance(c->ds, c->st, st));
@@ -693,8 +760,9 @@ nosa_status nosa_get_state(nosa_ctx* c, void* buf, size_t* size) {
   nosa_status s = set_device(c);
   if (s != NOSA_OK) return s;
   NOSA_CUDA(cudaDeviceSynchronize());
+  if ((s = flush_write_through(c)) != NOSA_OK) return s;
   unsigned char* p = static_cast<unsigned char*>(buf);
-  StateHeader h{kMagic, 1u, c->U, c->k, c->cfg.k_agnostic, c->C, c->max_blocks, c->G};
+  StateHeader h{kMagic, 2u, c->U, c->k, c->cfg.k_agnostic, c->C, c->max_blocks, c->G};
   memcpy(p, &h, sizeof h);
   p += sizeof h;
   const size_t U = c->U, KE = c->cfg.k_agnostic > 0 ? c->cfg.k_agnostic : 1;
@@ -727,24 +795,31 @@ nosa_status nosa_set_state(nosa_ctx* c, const void* buf, size_t size) {
   if (size != need) return fail(NOSA_ERR_INVALID, "state blob of %zu bytes, expected %zu", size, need);
   StateHeader h;
   memcpy(&h, buf, sizeof h);
-  if (h.magic != kMagic || h.version != 1u || h.U != c->U || h.k != c->k || h.k_e != c->cfg.k_agnostic ||
+  if (h.magic != kMagic || h.version != 2u || h.U != c->U || h.k != c->k || h.k_e != c->cfg.k_agnostic ||
       h.C != c->C || h.max_blocks != c->max_blocks || h.G != c->G)
     return fail(NOSA_ERR_INVALID, "state blob from a different configuration");
   nosa_status s = set_device(c);
   if (s != NOSA_OK) return s;
   NOSA_CUDA(cudaDeviceSynchronize());
+  if ((s = flush_write_through(c)) != NOSA_OK) return s;
   const unsigned char* p = static_cast<const unsigned char*>(buf) + sizeof h;
   DevState d;
   memcpy(&d, p, sizeof d);
   if (d.n_closed < 0 || d.n_closed > c->max_blocks || d.tail_len < 0 || d.tail_len >= kP)
     return fail(NOSA_ERR_INVALID, "state blob holds an invalid block count");
+  // the blob was taken after a write-through flush: every closed block is in
+  // the attached store and nothing is staged in this context
+  d.staged_block = -1;
+  d.wt_block = -1;
+  d.wt_done = 0;
   const size_t U = c->U, KE = c->cfg.k_agnostic > 0 ? c->cfg.k_agnostic : 1;
   auto put = [&](void* dev, size_t bytes) -> nosa_status {
     NOSA_CUDA(cudaMemcpy(dev, p, bytes, cudaMemcpyHostToDevice));
     p += bytes;
     return NOSA_OK;
   };
-  if ((s = put(c->ds, sizeof(DevState))) != NOSA_OK) return s;
+  NOSA_CUDA(cudaMemcpy(c->ds, &d, sizeof d, cudaMemcpyHostToDevice));
+  p += sizeof d;
   if ((s = put(c->ge, U * KE * 4)) != NOSA_OK) return s;
   if ((s = put(c->prev, U * c->k * 4)) != NOSA_OK) return s;
   if ((s = put(c->agnostic, U * c->max_blocks * 4)) != NOSA_OK) return s;

@@ -273,6 +273,9 @@ __device__ __forceinline__ uint4 ld_sys(const uint4* p) {
 
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
   const int count = *a.count;
+  // the most recently closed block may not have reached the host store yet:
+  // it is read from its staging copy in HBM
+  const int staged = a.stage_k ? a.ds->staged_block : -1;
   constexpr int kPer = kBlockBytes / 16 / kGatherThreads;  // 4 words of K (and of V) per thread
   for (int e = blockIdx.x; e < count; e += gridDim.x) {
     const int4 it = a.glist[e];
@@ -282,8 +285,10 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
     }
     const size_t src = ((size_t)it.x * a.max_blocks + it.y) * (kBlockBytes / 16);
     const size_t dst = ((size_t)it.x * a.C + it.z) * (kBlockBytes / 16);
-    const uint4* sk = reinterpret_cast<const uint4*>(a.hk) + src;
-    const uint4* sv = reinterpret_cast<const uint4*>(a.hv) + src;
+    const bool from_stage = it.y == staged;
+    const size_t s0 = from_stage ? (size_t)it.x * (kBlockBytes / 16) : src;
+    const uint4* sk = reinterpret_cast<const uint4*>(from_stage ? a.stage_k : a.hk) + s0;
+    const uint4* sv = reinterpret_cast<const uint4*>(from_stage ? a.stage_v : a.hv) + s0;
     uint4* dk = reinterpret_cast<uint4*>(a.ck) + dst;
     uint4* dv = reinterpret_cast<uint4*>(a.cv) + dst;
     uint4 rk[kPer], rv[kPer];

@@ -34,7 +34,10 @@ struct DevState {
   int tail_len_step;   // tail length during the step (tail_len + appended)
   int gather_count;    // entries in the gather list of the current step
   unsigned error_bits;
-  int pad;
+  int staged_block;    // closed block whose K/V sit in the staging buffer, -1 none
+  int wt_block;        // staged block not yet written through to the store, -1 none
+  int wt_done;         // CTAs of the write-through launch that have finished
+  int pad[2];
 };
 
 struct DevStats {
@@ -252,6 +255,8 @@ struct GatherArgs {
   uint16_t* cv;
   const int4* glist;
   const int* count;         // entries to copy (device)
+  const uint16_t* stage_k;  // [U, P, d] last closed block (null: nothing staged)
+  const uint16_t* stage_v;
   DevState* ds;
   int U, C, max_blocks;
 };
@@ -311,14 +316,31 @@ struct CloseArgs {
   float* agnostic;          // [U, max_blocks]
   uint16_t* kv_k;           // attached K (host mapped or device) [U, max_blocks*P, d]
   uint16_t* kv_v;
+  uint16_t* stage_k;        // [U, P, d] or null: the closed block goes to the store directly
+  uint16_t* stage_v;
   DevState* ds;
   int U, max_blocks;
 };
 cudaError_t launch_close(const CloseArgs& a, cudaStream_t st);
 
+struct WriteThroughArgs {
+  const uint16_t* stage_k;  // [U, P, d]
+  const uint16_t* stage_v;
+  uint16_t* kv_k;           // attached K in pinned host memory (device address)
+  uint16_t* kv_v;
+  DevState* ds;
+  int U, max_blocks;
+};
+// Low CTA priority; returns at once when no staged block is pending.
+cudaError_t launch_write_through(const WriteThroughArgs& a, int grid, cudaStream_t st);
+
 cudaError_t launch_advance(DevState* ds, DevStats* st, cudaStream_t s);
 // Sets the calling thread's nosa_last_error() message.
 void record_error(const char* msg);
+
+// Classify a pointer: 1 device (or managed) memory, 2 pinned or registered host
+// memory, whose device address is stored in *dev_ptr; 0 anything else.
+int pointer_kind(const void* p, void** dev_ptr);
 cudaError_t launch_init_state(DevState* ds, int n_closed, int tail_len, int step, int n_last_select,
                               cudaStream_t s);
 cudaError_t launch_reset_stats(DevStats* st, cudaStream_t s);

@@ -40,8 +40,12 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
 
 // ---------------------------------------------------------------- block close
 // When the tail holds P tokens at the end of a step, it becomes closed block
-// n: its pooled keys are built (same rule as at attach), its agnostic score is
-// registered, and K/V are written through to the attached KV store.
+// n: its pooled keys are built (same rule as at attach) and its agnostic score
+// is registered.  Its K/V go to the attached KV store directly when that store
+// is in HBM.  When the store is in host memory they go to a staging buffer in
+// HBM instead, and write_through_kernel moves them to the host during the next
+// step, off the critical path; until the next close the gather reads block n
+// from the staging copy.
 __global__ void __launch_bounds__(256) close_kernel(CloseArgs a) {
   const int u = blockIdx.x;
   if (a.ds->tail_len_step != kP) return;
@@ -71,18 +75,80 @@ __global__ void __launch_bounds__(256) close_kernel(CloseArgs a) {
     *kb = make_uint4(ob[0] | (ob[1] << 16), ob[2] | (ob[3] << 16), ob[4] | (ob[5] << 16),
                      ob[6] | (ob[7] << 16));
   }
-  uint4* dk = reinterpret_cast<uint4*>(a.kv_k) + ((size_t)u * a.max_blocks + n) * kP * kRowU4;
-  uint4* dv = reinterpret_cast<uint4*>(a.kv_v) + ((size_t)u * a.max_blocks + n) * kP * kRowU4;
+  const bool staged = a.stage_k != nullptr;
+  const size_t dst = staged ? (size_t)u * kP * kRowU4 : ((size_t)u * a.max_blocks + n) * kP * kRowU4;
+  uint4* dk = reinterpret_cast<uint4*>(staged ? a.stage_k : a.kv_k) + dst;
+  uint4* dv = reinterpret_cast<uint4*>(staged ? a.stage_v : a.kv_v) + dst;
   for (int i = threadIdx.x; i < kP * kRowU4; i += blockDim.x) {
     dk[i] = tk[i];
     dv[i] = tv[i];
   }
   if (threadIdx.x == 0) a.agnostic[(size_t)u * a.max_blocks + n] = a.a_pending[u];
+  if (staged && u == 0 && threadIdx.x == 0) {
+    a.ds->staged_block = n;
+    a.ds->wt_block = n;
+  }
 }
 
 cudaError_t launch_close(const CloseArgs& a, cudaStream_t st) {
   close_kernel<<<a.U, 256, 0, st>>>(a);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- write-through
+// Copies the staged block of every unit into the host KV store with
+// zero-copy stores (device-to-host over PCIe, the direction the miss gather
+// does not use).  The launch that finds a block pending clears the flag from
+// its last CTA; a launch with nothing pending returns at once.
+__global__ void __launch_bounds__(256) write_through_kernel(WriteThroughArgs a) {
+  const int n = a.ds->wt_block;
+  if (n < 0) return;
+  if (n >= a.max_blocks) {
+    if (threadIdx.x == 0) atomicOr(&a.ds->error_bits, ERR_RANGE);
+    return;
+  }
+  for (int u = blockIdx.x; u < a.U; u += gridDim.x) {
+    const uint4* sk = reinterpret_cast<const uint4*>(a.stage_k) + (size_t)u * kP * kRowU4;
+    const uint4* sv = reinterpret_cast<const uint4*>(a.stage_v) + (size_t)u * kP * kRowU4;
+    uint4* dk = reinterpret_cast<uint4*>(a.kv_k) + ((size_t)u * a.max_blocks + n) * kP * kRowU4;
+    uint4* dv = reinterpret_cast<uint4*>(a.kv_v) + ((size_t)u * a.max_blocks + n) * kP * kRowU4;
+    uint4 rk[kP * kRowU4 / 256], rv[kP * kRowU4 / 256];
+#pragma unroll
+    for (int i = 0; i < kP * kRowU4 / 256; ++i) {
+      rk[i] = sk[threadIdx.x + i * 256];
+      rv[i] = sv[threadIdx.x + i * 256];
+    }
+#pragma unroll
+    for (int i = 0; i < kP * kRowU4 / 256; ++i) {
+      dk[threadIdx.x + i * 256] = rk[i];
+      dv[threadIdx.x + i * 256] = rv[i];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence_system();
+    if (atomicAdd(&a.ds->wt_done, 1) == (int)gridDim.x - 1) {
+      a.ds->wt_block = -1;
+      a.ds->wt_done = 0;
+    }
+  }
+}
+
+cudaError_t launch_write_through(const WriteThroughArgs& a, int grid, cudaStream_t st) {
+  int least = 0, greatest = 0;
+  cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributePriority;
+  attr[0].val.priority = least;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, write_through_kernel, a);
 }
 
 // ---------------------------------------------------------------- step state
@@ -101,7 +167,10 @@ __global__ void init_state_kernel(DevState* ds, int n_closed, int tail_len, int 
   ds->tail_len_step = tail_len;
   ds->gather_count = 0;
   ds->error_bits = 0u;
-  ds->pad = 0;
+  ds->staged_block = -1;
+  ds->wt_block = -1;
+  ds->wt_done = 0;
+  ds->pad[0] = ds->pad[1] = 0;
 }
 
 cudaError_t launch_init_state(DevState* ds, int n_closed, int tail_len, int step, int n_last_select,

@@ -31,6 +31,7 @@ ENTRY_POINTS = (
     "nosa_select", "nosa_fetch_missing", "nosa_sparse_decode", "nosa_get_stats", "nosa_reset_stats",
     "nosa_check_errors", "nosa_read_cache_map", "nosa_get_state", "nosa_set_state",
     "nosa_debug_wait_flag", "nosa_last_error", "nosa_version", "nosa_sparse_decode_noalloc",
+    "nosa_gather_rows",
 )
 
 
@@ -91,6 +92,7 @@ def lib() -> C.CDLL:
             "nosa_last_error": ([], C.c_char_p),
             "nosa_version": ([], C.c_char_p),
             "nosa_sparse_decode_noalloc": ([vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp], st),
+            "nosa_gather_rows": ([vp, C.c_int64, vp, C.c_int64, i32, vp, vp, i32, i32, vp, vp], st),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -217,6 +219,13 @@ def nosa_sparse_decode_noalloc(q, k, v, batch: int, n_q_heads: int, n_kv_heads: 
     _check(lib().nosa_sparse_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), int(batch), int(n_q_heads),
                                             int(n_kv_heads), int(max_blocks), _ptr(sel), int(k_sel),
                                             _ptr(out), _stream(stream)), "nosa_sparse_decode_noalloc")
+
+
+def nosa_gather_rows(src, src_rows: int, dst, dst_rows: int, row_bytes: int, src_idx, dst_idx, n: int,
+                     ctas: int = 0, flags=None, stream=None) -> None:
+    _check(lib().nosa_gather_rows(_ptr(src), int(src_rows), _ptr(dst), int(dst_rows), int(row_bytes),
+                                  _ptr(src_idx), _ptr(dst_idx), int(n), int(ctas), _ptr(flags),
+                                  _stream(stream)), "nosa_gather_rows")
 
 
 def config_from_workload(w) -> nosa_config:

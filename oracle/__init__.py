@@ -212,6 +212,22 @@ class UnitRun:
     scores: Optional[np.ndarray]    # [steps, max_blocks]
 
 
+def gather_rows(src: np.ndarray, src_idx: Sequence[int], dst: np.ndarray,
+                dst_idx: Optional[Sequence[int]] = None) -> np.ndarray:
+    """Transfer of missed rows (NOSA summary §4: each miss is copied from host
+    memory into its GPU slot; §3.2: at block or at single-token granularity).
+    For each i in order, row dst_idx[i] (row i when dst_idx is None) of a copy
+    of dst takes row src_idx[i] of src; an index outside either array leaves
+    that row alone.  src and dst are 2-D arrays of one row width.  Returns the
+    updated copy."""
+    out = np.array(dst, copy=True)
+    for i, s in enumerate(src_idx):
+        t = i if dst_idx is None else dst_idx[i]
+        if 0 <= s < src.shape[0] and 0 <= t < out.shape[0]:
+            out[t, :] = src[s, :]
+    return out
+
+
 def make_cfg(G, d, P, Q, n0, tail0, max_blocks, k_q, k_e, m, C_slots, steps, append, sink=0,
              window=0) -> OrcCfg:
     return OrcCfg(G, d, P, Q, n0, tail0, max_blocks, k_q, k_e, m, C_slots, steps, int(append), sink, window)

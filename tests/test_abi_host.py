@@ -128,3 +128,24 @@ def test_every_workload_config_validates_host_side(L):
             L.nosa_destroy(out)
         else:
             assert rc in (nosa.NOSA_ERR_CUDA, nosa.NOSA_ERR_NOMEM), (name, nosa.nosa_last_error())
+
+
+@pytest.mark.parametrize("row_bytes,n,ctas", [(24, 1, 0), (8, 1, 0), (131072, 1, 0), (256, -1, 0),
+                                              (256, 1, -1), (256, 1, 70000)])
+def test_gather_rows_rejects_bad_sizes(L, row_bytes, n, ctas):
+    rc = L.nosa_gather_rows(None, 0, None, 0, row_bytes, None, None, n, ctas, None, None)
+    assert rc == nosa.NOSA_ERR_INVALID
+
+
+def test_gather_rows_with_no_rows_is_a_no_op(L):
+    assert L.nosa_gather_rows(None, 0, None, 0, 256, None, None, 0, 0, None, None) == nosa.NOSA_OK
+
+
+def test_gather_rows_rejects_pageable_memory(L):
+    import numpy as np
+    src = np.zeros((4, 64), dtype=np.uint32)     # pageable host memory
+    dst = np.zeros((4, 64), dtype=np.uint32)
+    idx = np.arange(4, dtype=np.int64)
+    with pytest.raises(nosa.NosaError) as e:
+        nosa.nosa_gather_rows(src, 4, dst, 4, 256, idx, None, 4)
+    assert e.value.status == nosa.NOSA_ERR_INVALID

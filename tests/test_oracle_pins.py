@@ -622,3 +622,34 @@ def test_block_leaving_the_window_joins_the_agnostic_pool(orc):
     for t in range(128, steps):
         assert 10 in r.sel[t].tolist()          # now through Gamma_e
         assert 11 in r.sel[t].tolist()          # the new window block
+
+
+# ---------------------------------------------------------------- row transfer
+
+def test_gather_rows_hand_example(orc):
+    """Rows move by their indices, source and destination not swapped."""
+    src = np.array([[1, 2], [3, 4], [5, 6]], dtype=np.uint8)
+    dst = np.zeros((4, 2), dtype=np.uint8)
+    got = orc.gather_rows(src, [2, 0], dst, [1, 3])
+    assert got.tolist() == [[0, 0], [5, 6], [0, 0], [1, 2]]
+    assert dst.sum() == 0  # the input is not modified
+    assert orc.gather_rows(src, [1, 2], dst).tolist() == [[3, 4], [5, 6], [0, 0], [0, 0]]
+
+
+def test_gather_rows_skips_out_of_range(orc):
+    src = np.arange(6, dtype=np.uint8).reshape(3, 2)
+    dst = np.full((2, 2), 9, dtype=np.uint8)
+    got = orc.gather_rows(src, [3, -1, 0], dst, [0, 1, 5])
+    assert got.tolist() == [[9, 9], [9, 9]]
+
+
+def test_block_rows_equal_their_token_rows(orc):
+    """A 64-token block row is the same bytes as its 64 token rows: moving a
+    block whole or token by token yields the same cache."""
+    rng = np.random.default_rng(3)
+    tok = rng.integers(0, 256, size=(4 * 64, 256), dtype=np.uint8)   # 4 blocks of 64 tokens
+    blk = tok.reshape(4, 64 * 256)
+    cache_b = orc.gather_rows(blk, [2, 0], np.zeros((2, 64 * 256), np.uint8))
+    tok_idx = [2 * 64 + i for i in range(64)] + [i for i in range(64)]
+    cache_t = orc.gather_rows(tok, tok_idx, np.zeros((128, 256), np.uint8))
+    assert np.array_equal(cache_b.reshape(128, 256), cache_t)
