@@ -340,7 +340,11 @@ def run_ours(args):
     # with appends also append, close and advance (otherwise the last
     # attention CTA ends the step), and with KV in host memory the
     # write-through of a block the previous step closed
-    launches_per_step = (6 if w.offloaded else 3) + (3 if w.append else 0) + (1 if w.append and w.offloaded else 0)
+    # (the fused entry point replaces score, select and plan by one kernel
+    # up to 512 blocks per unit)
+    fused = dec.fused and w.max_blocks <= 512
+    launches_per_step = ((4 if w.offloaded else 2) if fused else (6 if w.offloaded else 3)) \
+        + (3 if w.append else 0) + (1 if w.append and w.offloaded else 0)
     gather_ms = phase["gather_ms"]
     attn_ms = phase["attention_ms"]
     gather_gbs = (phase["fetched_bytes_per_step"] / (gather_ms * 1e-3) / 1e9) if gather_ms > 0 else 0.0
@@ -372,7 +376,11 @@ def run_ours(args):
                        "k_agnostic": w.k_agnostic, "min_overlap": w.min_overlap, "sink_blocks": w.sink_blocks,
                        "window_blocks": w.window_blocks, "cache_slots": w.cache_slots,
                        "kv": "pinned host" if w.offloaded else "HBM", "parallelism": f"replicas x{world}",
-                       "l2": "per-step traffic 288 MiB > 126 MB L2, no flush", "graph": "cuda graph replay"},
+                       "l2": (f"per-step HBM traffic {hbm_bytes / 2**20:.0f} MiB "
+                              + ("> 126 MB L2, no flush" if hbm_bytes > 126e6 else "< 126 MB L2, not flushed")),
+                       "graph": "cuda graph replay",
+                       "calls": ("nosa_score_select_fetch (fused) + nosa_sparse_decode" if fused
+                                 else "nosa_score_blocks + nosa_select + nosa_fetch_missing + nosa_sparse_decode")},
             "roofline": dominant,
             "roofline_other": other,
             "roofline_step": {
@@ -418,11 +426,17 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
         if w.append:
             nosa.nosa_append_token(dec.ctx, dec.k_in, dec.v_in, dec.a_in, s)
         ev["a"].record(s)
-        nosa.nosa_score_blocks(dec.ctx, dec.q, dec.scores, s)
-        ev["b"].record(s)
-        nosa.nosa_select(dec.ctx, dec.scores, dec.sel, s)
-        ev["c"].record(s)
-        nosa.nosa_fetch_missing(dec.ctx, dec.sel, dec.fetch, dec.n_fetch, s, cs)
+        if dec.fused:
+            # score, select and plan in one launch (b and c mark nothing)
+            nosa.nosa_score_select_fetch(dec.ctx, dec.q, dec.scores, dec.sel, dec.fetch, dec.n_fetch, s, cs)
+            ev["b"].record(s)
+            ev["c"].record(s)
+        else:
+            nosa.nosa_score_blocks(dec.ctx, dec.q, dec.scores, s)
+            ev["b"].record(s)
+            nosa.nosa_select(dec.ctx, dec.scores, dec.sel, s)
+            ev["c"].record(s)
+            nosa.nosa_fetch_missing(dec.ctx, dec.sel, dec.fetch, dec.n_fetch, s, cs)
         ev["d"].record(s)
         if cs is not s:
             ev["g"].record(cs)
@@ -432,7 +446,8 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
         else:
             s.wait_stream(cs)  # join the timing node recorded on the copy stream
         ev["e"].record(s)
-    acc = {"score_ms": 0.0, "select_ms": 0.0, "plan_ms": 0.0, "gather_ms": 0.0, "decode_ms": 0.0, "step_ms": 0.0}
+    acc = {"score_ms": 0.0, "select_ms": 0.0, "plan_ms": 0.0, "prepare_ms": 0.0, "gather_ms": 0.0,
+           "decode_ms": 0.0, "step_ms": 0.0}
     fb0 = dec.stats()["fetched_bytes"]
     for _ in range(n):
         t = dec.t
@@ -444,6 +459,7 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
         acc["score_ms"] += ev["a"].elapsed_time(ev["b"])
         acc["select_ms"] += ev["b"].elapsed_time(ev["c"])
         acc["plan_ms"] += ev["c"].elapsed_time(ev["d"])
+        acc["prepare_ms"] += ev["a"].elapsed_time(ev["d"])
         if cs is not s:
             acc["gather_ms"] += ev["d"].elapsed_time(ev["g"])
         acc["decode_ms"] += ev["d"].elapsed_time(ev["e"])
@@ -453,6 +469,10 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
     out["fetched_bytes_per_step"] = (dec.stats()["fetched_bytes"] - fb0) / n
     out["steps"] = n
     out["single_stream"] = bool(single_stream)
+    out["fused_prepare"] = bool(dec.fused)
+    if dec.fused:
+        for k in ("score_ms", "select_ms", "plan_ms"):
+            out.pop(k)
     return out
 
 

@@ -14,6 +14,8 @@
  *   nosa_sparse_decode  GQA attention over the selected blocks (App. A)
  *
  * plus nosa_append_token first when the sequence grows during decoding.
+ * nosa_score_select_fetch makes the first three calls in one (fused below
+ * 512 blocks per unit).
  *
  * Terms.  A unit is one (sequence b, KV head g), numbered u = b*n_kv_heads + g.
  * G = n_q_heads / n_kv_heads query heads share a KV head; query head h uses KV
@@ -191,6 +193,18 @@ NOSA_API nosa_status nosa_select(nosa_ctx* ctx, const double* scores, int32_t* s
  * copied: fetch is all -1 and n_fetch all 0. */
 NOSA_API nosa_status nosa_fetch_missing(nosa_ctx* ctx, const int32_t* sel, int32_t* fetch,
                                int32_t* n_fetch, nosa_stream_t compute, nosa_stream_t copy);
+
+/* nosa_score_blocks, nosa_select and nosa_fetch_missing in one call, with
+ * the same arguments, results and order rule (first call of a step, after an
+ * optional nosa_append_token); on return the step is ready for
+ * nosa_sparse_decode.  With max_blocks <= 512 the scores, the selection and
+ * the cache plan of each unit come from one kernel (one CTA per unit), so the
+ * miss gather starts after a single launch; scores, sel, fetch and n_fetch
+ * are bit-identical to those of the three calls.  With more blocks it makes
+ * the three calls itself. */
+NOSA_API nosa_status nosa_score_select_fetch(nosa_ctx* ctx, const void* q, double* scores, int32_t* sel,
+                                             int32_t* fetch, int32_t* n_fetch, nosa_stream_t compute,
+                                             nosa_stream_t copy);
 
 /* Block-sparse GQA attention (NOSA summary App. A): for each query head h of
  * unit u,  out_h = sum_t softmax_t(q_h . K_t / sqrt(d)) V_t  over the tokens of

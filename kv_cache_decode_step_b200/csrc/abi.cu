@@ -130,6 +130,7 @@ struct nosa_ctx {
   cudaEvent_t ev_wt_fork = nullptr, ev_wt_done = nullptr;
   bool wt_forked = false;
   int wt_grid = 18;
+  int prep_warps = 4;       // warps per CTA of the fused score/select/plan kernel
 };
 
 namespace {
@@ -286,6 +287,13 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   // link's bandwidth-delay product; more CTAs only queue system-memory
   // requests that slow the attention running beside the gather
   c->gather_grid = (sms + 3) / 4;
+  // fused score/select/plan: one CTA per unit; with few units, wider CTAs keep
+  // about 16 warps per SM scoring (4, 8 or 16 warps per CTA)
+  {
+    int w = 4;
+    while (w < 16 && c->U * w * 2 <= sms * 16) w *= 2;
+    c->prep_warps = w;
+  }
   if (const char* v = getenv("NOSA_GATHER_CTAS")) c->gather_grid = atoi(v) > 0 ? atoi(v) : c->gather_grid;
   // two persistent attention CTAs per SM, each over an equal share of the
   // (unit, block) positions; a unit's blocks span a few CTAs' shares
@@ -474,13 +482,9 @@ nosa_status nosa_append_token(nosa_ctx* c, const void* k_new, const void* v_new,
   return NOSA_OK;
 }
 
-nosa_status nosa_score_blocks(nosa_ctx* c, const void* q, double* scores, nosa_stream_t stream) {
-  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
-  if (!c->attached) return fail(NOSA_ERR_ORDER, "score before attach");
-  if (c->phase != kReady) return fail(NOSA_ERR_ORDER, "score must start a step (after decode or append)");
-  if (!q || !scores) return fail(NOSA_ERR_INVALID, "q and scores must be non-NULL");
-  nosa_status s = set_device(c);
-  if (s != NOSA_OK) return s;
+namespace {
+
+ScoreArgs score_args(const nosa_ctx* c, const void* q, double* scores) {
   ScoreArgs a{};
   a.q = static_cast<const uint16_t*>(q);
   a.kbar = c->kbar;
@@ -491,27 +495,10 @@ nosa_status nosa_score_blocks(nosa_ctx* c, const void* q, double* scores, nosa_s
   a.Hkv = c->cfg.n_kv_heads;
   a.G = c->G;
   a.max_blocks = c->max_blocks;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (c->stage_k && c->appends_enabled) {
-    // a block closed by the previous step goes to the host store while this
-    // step runs; nosa_sparse_decode joins it before the next close
-    NOSA_CUDA(cudaEventRecord(c->ev_wt_fork, st));
-    NOSA_CUDA(cudaStreamWaitEvent(c->wt_stream, c->ev_wt_fork, 0));
-    NOSA_CUDA(launch_write_through(write_through_args(c), c->wt_grid, c->wt_stream));
-    NOSA_CUDA(cudaEventRecord(c->ev_wt_done, c->wt_stream));
-    c->wt_forked = true;
-  }
-  NOSA_CUDA(launch_score(a, st));
-  c->phase = kScored;
-  return NOSA_OK;
+  return a;
 }
 
-nosa_status nosa_select(nosa_ctx* c, const double* scores, int32_t* sel, nosa_stream_t stream) {
-  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
-  if (c->phase != kScored) return fail(NOSA_ERR_ORDER, "select must follow score");
-  if (!scores || !sel) return fail(NOSA_ERR_INVALID, "scores and sel must be non-NULL");
-  nosa_status s = set_device(c);
-  if (s != NOSA_OK) return s;
+SelectArgs select_args(const nosa_ctx* c, const double* scores, int32_t* sel) {
   SelectArgs a{};
   a.agnostic = c->agnostic;
   a.scores = scores;
@@ -529,27 +516,10 @@ nosa_status nosa_select(nosa_ctx* c, const double* scores, int32_t* sel, nosa_st
   a.words = c->words;
   a.sink = c->cfg.sink_blocks;
   a.window = c->cfg.window_blocks;
-  NOSA_CUDA(launch_select(a, reinterpret_cast<cudaStream_t>(stream)));
-  c->phase = kSelected;
-  return NOSA_OK;
+  return a;
 }
 
-nosa_status nosa_fetch_missing(nosa_ctx* c, const int32_t* sel, int32_t* fetch, int32_t* n_fetch,
-                               nosa_stream_t compute, nosa_stream_t copy) {
-  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
-  if (c->phase != kSelected) return fail(NOSA_ERR_ORDER, "fetch must follow select");
-  if (!sel || !fetch || !n_fetch) return fail(NOSA_ERR_INVALID, "sel, fetch and n_fetch must be non-NULL");
-  nosa_status s = set_device(c);
-  if (s != NOSA_OK) return s;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(compute);
-  cudaStream_t xs = reinterpret_cast<cudaStream_t>(copy);
-  if (!c->offloaded) {
-    NOSA_CUDA(cudaMemsetAsync(fetch, 0xFF, (size_t)c->U * c->k * sizeof(int32_t), cs));
-    NOSA_CUDA(cudaMemsetAsync(n_fetch, 0, (size_t)c->U * sizeof(int32_t), cs));
-    c->gather_on_side = false;
-    c->phase = kFetched;
-    return NOSA_OK;
-  }
+PlanArgs plan_args(const nosa_ctx* c, const int32_t* sel, int32_t* fetch, int32_t* n_fetch) {
   PlanArgs p{};
   p.sel = sel;
   p.fetch = fetch;
@@ -567,7 +537,24 @@ nosa_status nosa_fetch_missing(nosa_ctx* c, const int32_t* sel, int32_t* fetch, 
   p.k = c->k;
   p.C = c->C;
   p.max_blocks = c->max_blocks;
-  NOSA_CUDA(launch_plan(p, cs));
+  return p;
+}
+
+// A block closed by the previous step goes to the host store while this step
+// runs; nosa_sparse_decode joins it before the next close.
+nosa_status fork_write_through(nosa_ctx* c, cudaStream_t st) {
+  if (!(c->stage_k && c->appends_enabled)) return NOSA_OK;
+  NOSA_CUDA(cudaEventRecord(c->ev_wt_fork, st));
+  NOSA_CUDA(cudaStreamWaitEvent(c->wt_stream, c->ev_wt_fork, 0));
+  NOSA_CUDA(launch_write_through(write_through_args(c), c->wt_grid, c->wt_stream));
+  NOSA_CUDA(cudaEventRecord(c->ev_wt_done, c->wt_stream));
+  c->wt_forked = true;
+  return NOSA_OK;
+}
+
+// The miss gather of the step, after the plan on cs: on xs (forked from cs by
+// an event) or on cs itself.
+nosa_status launch_step_gather(nosa_ctx* c, cudaStream_t cs, cudaStream_t xs) {
   GatherArgs g{};
   g.hk = c->kv_k;
   g.hv = c->kv_v;
@@ -589,6 +576,89 @@ nosa_status nosa_fetch_missing(nosa_ctx* c, const int32_t* sel, int32_t* fetch, 
     NOSA_CUDA(cudaEventRecord(c->ev_gather, xs));
   } else {
     NOSA_CUDA(launch_gather(g, c->gather_grid, cs));
+  }
+  return NOSA_OK;
+}
+
+}  // namespace
+
+nosa_status nosa_score_blocks(nosa_ctx* c, const void* q, double* scores, nosa_stream_t stream) {
+  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
+  if (!c->attached) return fail(NOSA_ERR_ORDER, "score before attach");
+  if (c->phase != kReady) return fail(NOSA_ERR_ORDER, "score must start a step (after decode or append)");
+  if (!q || !scores) return fail(NOSA_ERR_INVALID, "q and scores must be non-NULL");
+  nosa_status s = set_device(c);
+  if (s != NOSA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((s = fork_write_through(c, st)) != NOSA_OK) return s;
+  NOSA_CUDA(launch_score(score_args(c, q, scores), st));
+  c->phase = kScored;
+  return NOSA_OK;
+}
+
+nosa_status nosa_select(nosa_ctx* c, const double* scores, int32_t* sel, nosa_stream_t stream) {
+  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
+  if (c->phase != kScored) return fail(NOSA_ERR_ORDER, "select must follow score");
+  if (!scores || !sel) return fail(NOSA_ERR_INVALID, "scores and sel must be non-NULL");
+  nosa_status s = set_device(c);
+  if (s != NOSA_OK) return s;
+  NOSA_CUDA(launch_select(select_args(c, scores, sel), reinterpret_cast<cudaStream_t>(stream)));
+  c->phase = kSelected;
+  return NOSA_OK;
+}
+
+nosa_status nosa_fetch_missing(nosa_ctx* c, const int32_t* sel, int32_t* fetch, int32_t* n_fetch,
+                               nosa_stream_t compute, nosa_stream_t copy) {
+  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
+  if (c->phase != kSelected) return fail(NOSA_ERR_ORDER, "fetch must follow select");
+  if (!sel || !fetch || !n_fetch) return fail(NOSA_ERR_INVALID, "sel, fetch and n_fetch must be non-NULL");
+  nosa_status s = set_device(c);
+  if (s != NOSA_OK) return s;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(compute);
+  cudaStream_t xs = reinterpret_cast<cudaStream_t>(copy);
+  if (!c->offloaded) {
+    NOSA_CUDA(cudaMemsetAsync(fetch, 0xFF, (size_t)c->U * c->k * sizeof(int32_t), cs));
+    NOSA_CUDA(cudaMemsetAsync(n_fetch, 0, (size_t)c->U * sizeof(int32_t), cs));
+    c->gather_on_side = false;
+    c->phase = kFetched;
+    return NOSA_OK;
+  }
+  NOSA_CUDA(launch_plan(plan_args(c, sel, fetch, n_fetch), cs));
+  if ((s = launch_step_gather(c, cs, xs)) != NOSA_OK) return s;
+  c->phase = kFetched;
+  return NOSA_OK;
+}
+
+nosa_status nosa_score_select_fetch(nosa_ctx* c, const void* q, double* scores, int32_t* sel, int32_t* fetch,
+                                    int32_t* n_fetch, nosa_stream_t compute, nosa_stream_t copy) {
+  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
+  if (!c->attached) return fail(NOSA_ERR_ORDER, "score before attach");
+  if (c->phase != kReady) return fail(NOSA_ERR_ORDER, "score must start a step (after decode or append)");
+  if (!q || !scores || !sel || !fetch || !n_fetch)
+    return fail(NOSA_ERR_INVALID, "q, scores, sel, fetch and n_fetch must be non-NULL");
+  if (!prepare_supported(c->max_blocks)) {
+    // beyond the fused kernel's block count: the three calls in a row
+    nosa_status s = nosa_score_blocks(c, q, scores, compute);
+    if (s == NOSA_OK) s = nosa_select(c, scores, sel, compute);
+    if (s == NOSA_OK) s = nosa_fetch_missing(c, sel, fetch, n_fetch, compute, copy);
+    return s;
+  }
+  nosa_status s = set_device(c);
+  if (s != NOSA_OK) return s;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(compute);
+  cudaStream_t xs = reinterpret_cast<cudaStream_t>(copy);
+  if ((s = fork_write_through(c, cs)) != NOSA_OK) return s;
+  PrepareArgs a{};
+  a.sc = score_args(c, q, scores);
+  a.se = select_args(c, scores, sel);
+  a.pl = plan_args(c, sel, fetch, n_fetch);
+  a.offloaded = c->offloaded ? 1 : 0;
+  a.nwarps = c->prep_warps;
+  NOSA_CUDA(launch_prepare(a, cs));
+  if (c->offloaded) {
+    if ((s = launch_step_gather(c, cs, xs)) != NOSA_OK) return s;
+  } else {
+    c->gather_on_side = false;
   }
   c->phase = kFetched;
   return NOSA_OK;

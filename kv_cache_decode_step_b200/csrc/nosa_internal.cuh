@@ -153,6 +153,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// 4-byte asynchronous copy global -> shared (completes at cp_async_wait_all).
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ double bf16_lo_to_f64(uint32_t w) { return (double)__uint_as_float(w << 16); }
 __device__ __forceinline__ double bf16_hi_to_f64(uint32_t w) {
   return (double)__uint_as_float(w & 0xFFFF0000u);
@@ -196,6 +202,7 @@ __device__ __forceinline__ void advance_step(DevState* ds, DevStats* st) {
     ds->tail_len = tl;
   }
   ds->tail_len_step = ds->tail_len;
+  ds->gather_count = 0;
   ds->step += 1;
   st->steps += 1;
 }
@@ -247,6 +254,21 @@ struct PlanArgs {
   int U, k, C, max_blocks;
 };
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st);
+
+// Score, selection and plan of each unit in one launch (one CTA per unit);
+// for max_blocks <= kPrepareMaxBlocks.  Needs gather_count = 0 on entry,
+// which every step's end leaves behind.
+constexpr int kPrepareMaxBlocks = 512;
+struct PrepareArgs {
+  ScoreArgs sc;
+  SelectArgs se;
+  PlanArgs pl;              // with KV resident only fetch / n_fetch are used
+  int offloaded;
+  int nwarps;               // warps per CTA (4..16): more when there are few units
+  int plan_ints;            // set by the launcher
+};
+bool prepare_supported(int max_blocks);
+cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t st);
 
 struct GatherArgs {
   const uint16_t* hk;       // host K (device-addressable), [U, max_blocks*P, d]

@@ -1,0 +1,106 @@
+// prepare.cu -- the first three stages of a decode step fused into one
+// kernel: block scores, selection and the cache plan of each unit.
+//
+// NOSA: Native and Offloadable Sparse Attention (paperlayer summary): §3.1
+// (scores from pooled keys; query-aware and query-agnostic selection under a
+// minimum overlap), §4 (set difference against the GPU-resident blocks and a
+// replacement mapping).  The arithmetic is that of score_kernel,
+// select_reg_kernel and the planning kernels: the same device functions run
+// here, only the launch boundaries between them are gone.  One CTA owns one
+// unit: its four warps score every closed block (scores kept in shared
+// memory), then warp 0 selects and plans.  The gather can start as soon as
+// this single launch ends instead of after three launches in a row.
+#include "plan_dev.cuh"
+#include "score_dev.cuh"
+#include "select_dev.cuh"
+
+namespace nosa {
+
+constexpr int kPrepMaxThreads = 512;
+
+// Shared memory: scores [max_blocks] fp64, selection bitmaps [2][R] words,
+// plan scratch (max(32, 2C + 2k) ints), then copies of the unit's S(t-1) [k],
+// Gamma_e(t-1) [k_e], the new selection [k], the register plan's slot tables
+// [32] x 2 and the general plan's block -> slot table [max_blocks].  The
+// copies are loaded while the scores stream in, so selection and planning
+// read no global memory of their own.
+template <int R>
+__global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs a) {
+  extern __shared__ __align__(16) unsigned char prep_smem[];
+  const int k = a.se.k, ke = a.se.k_e, C = a.pl.C;
+  double* ssc = reinterpret_cast<double*>(prep_smem);
+  unsigned(*sbm)[R] = reinterpret_cast<unsigned(*)[R]>(ssc + a.sc.max_blocks);
+  int* psm = reinterpret_cast<int*>(sbm + 2);
+  int* s_prev = psm + a.plan_ints;
+  int* s_ge = s_prev + k;
+  int* s_sel = s_ge + ke;
+  int* s_sb = s_sel + k;
+  int* s_lu = s_sb + 32;
+  int* s_bs = s_lu + 32;  // general plan: the unit's block -> slot table [max_blocks]
+  const int u = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool reg_plan = a.offloaded && C <= 32 && k <= 32;
+
+  // asynchronous copies: they land while the scores stream in
+  for (int i = threadIdx.x; i < k; i += blockDim.x) cp_async4(s_prev + i, a.se.prev + (size_t)u * k + i);
+  for (int i = threadIdx.x; i < ke; i += blockDim.x) cp_async4(s_ge + i, a.se.ge + (size_t)u * ke + i);
+  if (reg_plan) {
+    for (int i = threadIdx.x; i < C; i += blockDim.x) {
+      cp_async4(s_sb + i, a.pl.slot_block + (size_t)u * C + i);
+      cp_async4(s_lu + i, a.pl.last_used + (size_t)u * C + i);
+    }
+  } else if (a.offloaded) {
+    // the general plan's slot tables go where it keeps them (psm)
+    for (int i = threadIdx.x; i < C; i += blockDim.x) {
+      cp_async4(psm + i, a.pl.slot_block + (size_t)u * C + i);
+      cp_async4(psm + C + i, a.pl.last_used + (size_t)u * C + i);
+    }
+    for (int i = threadIdx.x; i < a.pl.max_blocks; i += blockDim.x)
+      cp_async4(s_bs + i, a.pl.block_slot + (size_t)u * a.pl.max_blocks + i);
+  }
+
+  score_unit_warps(a.sc, u, warp, blockDim.x >> 5, lane, ssc);
+  cp_async_wait_all();
+  __syncthreads();
+  if (warp != 0) return;
+
+  select_unit_reg<R>(a.se, u, lane, sbm, ssc, s_prev, s_ge, s_sel);
+  __syncwarp();  // the selection is read back by the plan
+
+  if (reg_plan) {
+    plan_unit_reg(a.pl, u, lane, psm, s_sel, s_sb, s_lu);
+  } else if (a.offloaded) {
+    plan_unit_smem(a.pl, u, lane, psm, s_sel, s_bs, true);
+  } else {
+    for (int i = lane; i < k; i += 32) a.pl.fetch[(size_t)u * k + i] = -1;
+    if (lane == 0) a.pl.n_fetch[u] = 0;
+  }
+}
+
+template <int R>
+cudaError_t launch_prepare_r(PrepareArgs a, cudaStream_t st) {
+  a.plan_ints = a.offloaded ? max(32, 2 * a.pl.C + 2 * a.pl.k) : 0;
+  const size_t smem = (size_t)a.sc.max_blocks * sizeof(double) + 2 * R * sizeof(unsigned) +
+                      (size_t)(a.plan_ints + 2 * a.se.k + a.se.k_e + 64) * sizeof(int) +
+                      (a.offloaded ? (size_t)a.pl.max_blocks * sizeof(int) : 0);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(prepare_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  const int threads = 32 * max(4, min(a.nwarps, kPrepMaxThreads / 32));
+  prepare_kernel<R><<<a.sc.U, threads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+bool prepare_supported(int max_blocks) { return max_blocks <= kPrepareMaxBlocks; }
+
+cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t st) {
+  const int rows = (a.sc.max_blocks + 31) / 32;
+  if (rows <= 2) return launch_prepare_r<2>(a, st);
+  if (rows <= 4) return launch_prepare_r<4>(a, st);
+  if (rows <= 8) return launch_prepare_r<8>(a, st);
+  if (rows <= 16) return launch_prepare_r<16>(a, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace nosa

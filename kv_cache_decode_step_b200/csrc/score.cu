@@ -5,7 +5,7 @@
 // pooling over the sub-blocks of a block.  Here a sub-block is 16 tokens and a
 // block 64 (4 sub-blocks); the sub-block score of KV head g sums the raw dot
 // products of its G query heads with the pooled key.
-#include "nosa_internal.cuh"
+#include "score_dev.cuh"
 
 namespace nosa {
 
@@ -67,31 +67,7 @@ cudaError_t launch_pool(const uint16_t* src, size_t src_unit_tokens, int U, int 
 constexpr int kScoreCtaBlocks = 32;
 constexpr int kScoreWarps = 4;
 constexpr int kScoreWarpBlocks = kScoreCtaBlocks / kScoreWarps;
-constexpr int kBlockU4 = kR * kRowU4;  // 16-byte words of pooled keys per block (64)
 constexpr uint64_t kScoreWaitNs = 1000000000ull;
-
-__device__ __forceinline__ double dot16(const uint4& a, const uint4& b, const double* qt) {
-  double s = 0.0;
-  s = fma(qt[0], bf16_lo_to_f64(a.x), s);  s = fma(qt[1], bf16_hi_to_f64(a.x), s);
-  s = fma(qt[2], bf16_lo_to_f64(a.y), s);  s = fma(qt[3], bf16_hi_to_f64(a.y), s);
-  s = fma(qt[4], bf16_lo_to_f64(a.z), s);  s = fma(qt[5], bf16_hi_to_f64(a.z), s);
-  s = fma(qt[6], bf16_lo_to_f64(a.w), s);  s = fma(qt[7], bf16_hi_to_f64(a.w), s);
-  s = fma(qt[8], bf16_lo_to_f64(b.x), s);  s = fma(qt[9], bf16_hi_to_f64(b.x), s);
-  s = fma(qt[10], bf16_lo_to_f64(b.y), s); s = fma(qt[11], bf16_hi_to_f64(b.y), s);
-  s = fma(qt[12], bf16_lo_to_f64(b.z), s); s = fma(qt[13], bf16_hi_to_f64(b.z), s);
-  s = fma(qt[14], bf16_lo_to_f64(b.w), s); s = fma(qt[15], bf16_hi_to_f64(b.w), s);
-  return s;
-}
-
-__device__ __forceinline__ double block_reduce(double s) {
-  s += __shfl_xor_sync(0xffffffffu, s, 1);
-  s += __shfl_xor_sync(0xffffffffu, s, 2);
-  s += __shfl_xor_sync(0xffffffffu, s, 4);
-  double o = __shfl_xor_sync(0xffffffffu, s, 8);
-  s = o > s ? o : s;
-  o = __shfl_xor_sync(0xffffffffu, s, 16);
-  return o > s ? o : s;
-}
 
 __global__ void __launch_bounds__(kScoreWarps * 32) score_kernel(ScoreArgs a) {
   __shared__ __align__(128) uint4 skb[kScoreCtaBlocks * kBlockU4];  // 32 KiB
@@ -120,18 +96,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32) score_kernel(ScoreArgs a) {
   const int r = lane >> 3, c = lane & 7;
   const int b = u / a.Hkv, g = u % a.Hkv;
   double qt[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) qt[i] = 0.0;
-  const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + (size_t)g * a.G) * kD);
-  for (int h = 0; h < a.G; ++h) {
-    const uint4 y0 = qrow[h * kRowU4 + c], y1 = qrow[h * kRowU4 + 8 + c];
-    const uint32_t wv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      qt[2 * i] += bf16_lo_to_f64(wv[i]);
-      qt[2 * i + 1] += bf16_hi_to_f64(wv[i]);
-    }
-  }
+  group_query_sum(a, b, g, c, qt);
 
   const int jw = warp * kScoreWarpBlocks;
   const int cnt = min(kScoreWarpBlocks, nb - jw);

@@ -31,7 +31,7 @@ ENTRY_POINTS = (
     "nosa_select", "nosa_fetch_missing", "nosa_sparse_decode", "nosa_get_stats", "nosa_reset_stats",
     "nosa_check_errors", "nosa_read_cache_map", "nosa_get_state", "nosa_set_state",
     "nosa_debug_wait_flag", "nosa_last_error", "nosa_version", "nosa_sparse_decode_noalloc",
-    "nosa_gather_rows",
+    "nosa_gather_rows", "nosa_score_select_fetch",
 )
 
 
@@ -93,6 +93,7 @@ def lib() -> C.CDLL:
             "nosa_version": ([], C.c_char_p),
             "nosa_sparse_decode_noalloc": ([vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp], st),
             "nosa_gather_rows": ([vp, C.c_int64, vp, C.c_int64, i32, vp, vp, i32, i32, vp, vp], st),
+            "nosa_score_select_fetch": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -171,6 +172,12 @@ def nosa_select(ctx, scores, sel, stream=None) -> None:
 def nosa_fetch_missing(ctx, sel, fetch, n_fetch, compute=None, copy=None) -> None:
     _check(lib().nosa_fetch_missing(ctx, _ptr(sel), _ptr(fetch), _ptr(n_fetch), _stream(compute),
                                     _stream(copy)), "nosa_fetch_missing")
+
+
+def nosa_score_select_fetch(ctx, q, scores, sel, fetch, n_fetch, compute=None, copy=None) -> None:
+    _check(lib().nosa_score_select_fetch(ctx, _ptr(q), _ptr(scores), _ptr(sel), _ptr(fetch), _ptr(n_fetch),
+                                         _stream(compute), _stream(copy if copy is not None else compute)),
+           "nosa_score_select_fetch")
 
 
 def nosa_sparse_decode(ctx, q, sel, out, stream=None) -> None:

@@ -30,8 +30,9 @@ class Decoder:
     """
 
     def __init__(self, w: Workload, data: Dict[str, np.ndarray], device: int = 0,
-                 side_copy_stream: bool = True, pin: bool = True):
+                 side_copy_stream: bool = True, pin: bool = True, fused: bool = True):
         self.w = w
+        self.fused = fused  # nosa_score_select_fetch instead of the three calls
         self.dev = torch.device("cuda", device)
         torch.cuda.set_device(self.dev)
         U, d = w.units, w.head_dim
@@ -118,9 +119,12 @@ class Decoder:
         s, cs = self.stream, self.copy_stream
         if append:
             nosa.nosa_append_token(self.ctx, self.k_in, self.v_in, self.a_in, s)
-        nosa.nosa_score_blocks(self.ctx, self.q, self.scores, s)
-        nosa.nosa_select(self.ctx, self.scores, self.sel, s)
-        nosa.nosa_fetch_missing(self.ctx, self.sel, self.fetch, self.n_fetch, s, cs)
+        if self.fused:
+            nosa.nosa_score_select_fetch(self.ctx, self.q, self.scores, self.sel, self.fetch, self.n_fetch, s, cs)
+        else:
+            nosa.nosa_score_blocks(self.ctx, self.q, self.scores, s)
+            nosa.nosa_select(self.ctx, self.scores, self.sel, s)
+            nosa.nosa_fetch_missing(self.ctx, self.sel, self.fetch, self.n_fetch, s, cs)
         nosa.nosa_sparse_decode(self.ctx, self.q, self.sel, self.out, s)
 
     def step(self) -> None:

@@ -29,10 +29,10 @@ class GpuRecord:
 
 
 def run_gpu(w, data, sample: Sequence[int], attend_steps, steps=None, graph=False,
-            cache_steps=(), side_copy_stream=True) -> GpuRecord:
+            cache_steps=(), side_copy_stream=True, fused=True) -> GpuRecord:
     steps = w.steps if steps is None else steps
     sample = list(sample)
-    dec = runner.Decoder(w, data, side_copy_stream=side_copy_stream)
+    dec = runner.Decoder(w, data, side_copy_stream=side_copy_stream, fused=fused)
     rec = GpuRecord(sel=np.zeros((steps, len(sample), w.k), np.int32),
                     fetch=np.zeros((steps, len(sample), w.k), np.int32),
                     nfetch=np.zeros((steps, len(sample)), np.int32))

@@ -113,3 +113,33 @@ def test_side_stream_and_single_stream_agree():
     assert np.array_equal(a.sel, b.sel) and np.array_equal(a.fetch, b.fetch)
     for t in a.out:
         assert np.array_equal(a.out[t], b.out[t])
+
+
+# ------------------------------------------------------------------ fused entry point
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", {}),
+    ("tiny", {"offloaded": False, "cache_factor": 0}),
+    ("layer8b", {"batch": 4, "steps": 24}),
+    ("offload_b64", {"steps": 24}),
+    ("long_gen", {"batch": 2, "steps": 70}),
+    ("long_input", {"batch": 1, "steps": 6}),   # beyond the fused kernel: three calls
+])
+@pytest.mark.parametrize("graph", [False, True])
+def test_fused_and_separate_calls_agree_bit_exactly(name, kw, graph):
+    """nosa_score_select_fetch gives the selections, fetch lists, outputs and
+    statistics of score + select + fetch, bit for bit (same arithmetic)."""
+    w = configs.get(name, **kw)
+    data = inputs.generate(w)
+    sample = list(range(min(w.units, 8)))
+    attend = list(range(w.steps))
+    a = run_gpu(w, data, sample, attend, graph=graph, cache_steps=[w.steps - 1], fused=True)
+    b = run_gpu(w, data, sample, attend, graph=graph, cache_steps=[w.steps - 1], fused=False)
+    assert np.array_equal(a.sel, b.sel) and np.array_equal(a.fetch, b.fetch)
+    assert np.array_equal(a.nfetch, b.nfetch) and np.array_equal(a.sel_all_last, b.sel_all_last)
+    for t in attend:
+        assert np.array_equal(a.out[t], b.out[t]), t
+    for t in a.resident:
+        for x, y in zip(a.resident[t], b.resident[t]):
+            assert np.array_equal(x, y)
+    assert a.stats == b.stats
