@@ -326,9 +326,10 @@ def run_ours(args):
     phase1 = instrumented_pass(torch, dec, w, nosa, n=min(args.steps, 50), single_stream=True)
     phase["attention_ms"] = phase1["decode_ms"]
     phase["single_stream_step_ms"] = phase1["step_ms"]
-    phase["note"] = ("graph-captured step with timing events between the ABI calls; gather_ms from the "
-                     "side-stream pass, attention_ms (both attention launches + combine + advance) from a "
-                     "single-stream pass where the gather has finished before attention starts")
+    phase["note"] = ("graph-captured step with timing events between the ABI calls; gather_ms (the fused "
+                     "gather + miss attention, from the end of the plan) from the side-stream pass; "
+                     "attention_ms = the decode call of a single-stream pass (KV in HBM: the hits pass; KV in "
+                     "host memory: the gather + miss attention, then the hits pass)")
 
     latency = step_latency_pass(torch, dec, w, LATENCY_STEPS)
 
@@ -336,28 +337,32 @@ def run_ours(args):
     e2e = e2e_pass(torch, dec, w, nosa, args.e2e_steps)
     e2e["eager_value"] = e2e_pass(torch, dec, w, nosa, args.e2e_steps, eager=True)["value"]
 
-    # kernels per step: score, select, [plan, gather, misses pass], hits pass;
-    # with appends also append, close and advance (otherwise the last
-    # attention CTA ends the step), and with KV in host memory the
-    # write-through of a block the previous step closed
-    # (the fused entry point replaces score, select and plan by one kernel
-    # up to 512 blocks per unit)
+    # kernels per step: score, select, [plan, gather + miss attention], hits
+    # pass -- the fused entry point makes score, select and plan one kernel up
+    # to 512 blocks per unit; with appends also append, close and advance
+    # (otherwise the last unit merged ends the step), and with KV in host
+    # memory the write-through of a block the previous step closed
     fused = dec.fused and w.max_blocks <= 512
-    launches_per_step = ((4 if w.offloaded else 2) if fused else (6 if w.offloaded else 3)) \
+    launches_per_step = ((3 if w.offloaded else 2) if fused else (5 if w.offloaded else 3)) \
         + (3 if w.append else 0) + (1 if w.append and w.offloaded else 0)
     gather_ms = phase["gather_ms"]
     attn_ms = phase["attention_ms"]
     gather_gbs = (phase["fetched_bytes_per_step"] / (gather_ms * 1e-3) / 1e9) if gather_ms > 0 else 0.0
     attn_bytes = w.units * w.k * w.block * w.head_dim * 2 * 2 + w.batch * w.n_q_heads * w.head_dim * 2 * 2
     attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9 if attn_ms > 0 else 0.0
-    rl_gather = {"kernel": "gather_kernel", "bound": "pcie", "achieved": gather_gbs, "peak": h2d_peak,
+    rl_gather = {"kernel": "gather_attend_kernel", "bound": "pcie", "achieved": gather_gbs, "peak": h2d_peak,
                  "unit": "GB/s", "frac": gather_gbs / h2d_peak if h2d_peak else None, "traffic": None,
                  "peak_source": "pinned cudaMemcpyAsync H2D measured in this run (256 MiB)",
                  "bytes_per_launch": phase["fetched_bytes_per_step"], "ms_per_launch": gather_ms}
-    rl_attn = {"kernel": "decode_kernel x2 + combine_kernel + advance_kernel", "bound": "hbm", "achieved": attn_gbs,
+    rl_attn = {"kernel": "attend_hits_kernel", "bound": "hbm", "achieved": attn_gbs,
                "peak": hbm_meas, "unit": "GB/s", "frac": attn_gbs / hbm_meas, "traffic": None,
                "peak_source": f"hbm_gbs {hbm_src}", "bytes_per_launch": attn_bytes, "ms_per_launch": attn_ms}
-    dominant, other = (rl_gather, rl_attn) if gather_ms >= attn_ms else (rl_attn, rl_gather)
+    if w.offloaded:
+        # the hits pass runs beside the gather (and, on one stream, after it):
+        # its own duration is not separable from the step's events
+        dominant, other = rl_gather, None
+    else:
+        dominant, other = rl_attn, None
 
     result = None
     if rank == 0:
@@ -438,12 +443,11 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
             ev["c"].record(s)
             nosa.nosa_fetch_missing(dec.ctx, dec.sel, dec.fetch, dec.n_fetch, s, cs)
         ev["d"].record(s)
-        if cs is not s:
-            ev["g"].record(cs)
+        # the decode call launches the fused gather + miss attention on the copy
+        # stream beside the hits pass: g marks its end
         nosa.nosa_sparse_decode(dec.ctx, dec.q, dec.sel, dec.out, s)
-        if cs is s:
-            ev["g"].record(s)
-        else:
+        ev["g"].record(cs)
+        if cs is not s:
             s.wait_stream(cs)  # join the timing node recorded on the copy stream
         ev["e"].record(s)
     acc = {"score_ms": 0.0, "select_ms": 0.0, "plan_ms": 0.0, "prepare_ms": 0.0, "gather_ms": 0.0,
@@ -460,7 +464,7 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
         acc["select_ms"] += ev["b"].elapsed_time(ev["c"])
         acc["plan_ms"] += ev["c"].elapsed_time(ev["d"])
         acc["prepare_ms"] += ev["a"].elapsed_time(ev["d"])
-        if cs is not s:
+        if cs is not s and w.offloaded:
             acc["gather_ms"] += ev["d"].elapsed_time(ev["g"])
         acc["decode_ms"] += ev["d"].elapsed_time(ev["e"])
         acc["step_ms"] += ev["a"].elapsed_time(ev["e"])

@@ -183,14 +183,16 @@ NOSA_API nosa_status nosa_select(nosa_ctx* ctx, const double* scores, int32_t* s
  * misses M = S(t) \ R(t-1) (R = blocks resident in the GPU cache) get slots:
  * free slots first (lowest first), then resident blocks outside S(t), least
  * recently selected first, lower block id on ties.  Only blocks unused by this
- * step are replaced.  The K and V of each miss (2 x 16 KiB) are then copied
- * from pinned host memory into its slot by a zero-copy gather kernel.
- * sel: device int32 [U, k] from nosa_select.  fetch: device int32 [U, k], the
- * missed block ids ascending, -1 padded.  n_fetch: device int32 [U].
- * Planning runs on compute; the gather on copy, which may equal compute.  A
- * separate copy stream lets nosa_sparse_decode attend to the hit blocks while
- * the misses are in flight.  With KV resident (cache_slots = 0) nothing is
- * copied: fetch is all -1 and n_fetch all 0. */
+ * step are replaced.  sel: device int32 [U, k] from nosa_select.  fetch:
+ * device int32 [U, k], the missed block ids ascending, -1 padded.  n_fetch:
+ * device int32 [U].  Planning runs on compute, and the slot tables
+ * (nosa_read_cache_map) are final when it has run.  The copies themselves --
+ * K and V of each miss, 2 x 16 KiB, from pinned host memory into its slot by
+ * a zero-copy gather kernel that also attends to each block as it lands --
+ * are issued by nosa_sparse_decode on `copy`, which may equal compute; a
+ * separate copy stream lets the attention to the blocks already cached run
+ * beside the transfer.  With KV resident (cache_slots = 0) nothing is copied:
+ * fetch is all -1 and n_fetch all 0. */
 NOSA_API nosa_status nosa_fetch_missing(nosa_ctx* ctx, const int32_t* sel, int32_t* fetch,
                                int32_t* n_fetch, nosa_stream_t compute, nosa_stream_t copy);
 
@@ -210,8 +212,10 @@ NOSA_API nosa_status nosa_score_select_fetch(nosa_ctx* ctx, const void* q, doubl
  * unit u,  out_h = sum_t softmax_t(q_h . K_t / sqrt(d)) V_t  over the tokens of
  * the selected blocks plus the open tail, in fp32 with bf16 inputs; written as
  * bf16.  q: device bf16 [B, H_q, d]; sel: the same buffer passed to
- * nosa_select; out: device bf16 [B, H_q, d].  Ends the step: closes a full
- * tail block and advances the step counter. */
+ * nosa_select; out: device bf16 [B, H_q, d].  With KV in host memory it also
+ * issues the miss gather planned by the fetch call, on that call's copy
+ * stream (joined back into `stream` before it returns).  Ends the step:
+ * closes a full tail block and advances the step counter. */
 NOSA_API nosa_status nosa_sparse_decode(nosa_ctx* ctx, const void* q, const int32_t* sel, void* out,
                                nosa_stream_t stream);
 

@@ -111,13 +111,14 @@ struct nosa_ctx {
   bool maps_main = false;
   cudaEvent_t ev_plan = nullptr, ev_gather = nullptr;
   bool gather_on_side = false;
+  cudaStream_t copy_stream = nullptr;  // given to the fetch call; the decode call gathers on it
 
   // host mirror of the device step state (validation only)
   int h_n_closed = 0, h_tail = 0;
   bool h_appended = false, appends_enabled = false;
   Phase phase = kReady;
 
-  int nparts = 2, gather_grid = 148, attn_grid = 296;
+  int nparts = 2, hits_parts = 2, gather_grid = 148, attn_grid = 296;
   int* unit_done = nullptr;
   int* done_ctr = nullptr;
 
@@ -300,7 +301,9 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   int want = 2 * sms;
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
   c->attn_grid = attend_hits_grid(c->U, c->k, 1, want);
-  c->nparts = attend_hits_parts(c->U, c->k, 1, c->attn_grid);
+  c->hits_parts = attend_hits_parts(c->U, c->k, 1, c->attn_grid);
+  // partial slots per unit: the hits pass's segments, then one per fetched block
+  c->nparts = c->hits_parts + (c->offloaded ? c->k : 0);
 
   const size_t U = c->U, MB = c->max_blocks, K = c->k;
 #define ALLOC(ptr, n)                    \
@@ -552,34 +555,6 @@ nosa_status fork_write_through(nosa_ctx* c, cudaStream_t st) {
   return NOSA_OK;
 }
 
-// The miss gather of the step, after the plan on cs: on xs (forked from cs by
-// an event) or on cs itself.
-nosa_status launch_step_gather(nosa_ctx* c, cudaStream_t cs, cudaStream_t xs) {
-  GatherArgs g{};
-  g.hk = c->kv_k;
-  g.hv = c->kv_v;
-  g.ck = c->cache_k;
-  g.cv = c->cache_v;
-  g.glist = c->glist;
-  g.count = &c->ds->gather_count;
-  g.stage_k = c->stage_k;
-  g.stage_v = c->stage_v;
-  g.ds = c->ds;
-  g.U = c->U;
-  g.C = c->C;
-  g.max_blocks = c->max_blocks;
-  c->gather_on_side = (xs != cs);
-  if (c->gather_on_side) {
-    NOSA_CUDA(cudaEventRecord(c->ev_plan, cs));
-    NOSA_CUDA(cudaStreamWaitEvent(xs, c->ev_plan, 0));
-    NOSA_CUDA(launch_gather(g, c->gather_grid, xs));
-    NOSA_CUDA(cudaEventRecord(c->ev_gather, xs));
-  } else {
-    NOSA_CUDA(launch_gather(g, c->gather_grid, cs));
-  }
-  return NOSA_OK;
-}
-
 }  // namespace
 
 nosa_status nosa_score_blocks(nosa_ctx* c, const void* q, double* scores, nosa_stream_t stream) {
@@ -624,7 +599,8 @@ nosa_status nosa_fetch_missing(nosa_ctx* c, const int32_t* sel, int32_t* fetch, 
     return NOSA_OK;
   }
   NOSA_CUDA(launch_plan(plan_args(c, sel, fetch, n_fetch), cs));
-  if ((s = launch_step_gather(c, cs, xs)) != NOSA_OK) return s;
+  c->copy_stream = xs;
+  c->gather_on_side = (xs != cs);
   c->phase = kFetched;
   return NOSA_OK;
 }
@@ -655,11 +631,8 @@ nosa_status nosa_score_select_fetch(nosa_ctx* c, const void* q, double* scores, 
   a.offloaded = c->offloaded ? 1 : 0;
   a.nwarps = c->prep_warps;
   NOSA_CUDA(launch_prepare(a, cs));
-  if (c->offloaded) {
-    if ((s = launch_step_gather(c, cs, xs)) != NOSA_OK) return s;
-  } else {
-    c->gather_on_side = false;
-  }
+  c->copy_stream = xs;
+  c->gather_on_side = c->offloaded && xs != cs;
   c->phase = kFetched;
   return NOSA_OK;
 }
@@ -695,23 +668,44 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
   a.hits_grid = c->attn_grid;
   a.out = static_cast<uint16_t*>(out);
   a.st = c->st;
-  // Without a block close to follow, the last CTA of the step's last kernel
-  // ends the step itself (one launch fewer).
+  a.miss_base = c->hits_parts;
+  // Every unit's partials are counted in unit_done; whichever kernel completes
+  // a unit merges it, and without a block close to follow, the last unit
+  // merged ends the step itself (no advance launch).
   const bool fold_advance = !c->appends_enabled;
-  // hits pass: blocks already on the GPU (all of S(t) when KV is in HBM) plus
-  // the open tail; it overlaps the gather running on the copy stream.  With
-  // KV in HBM the last CTA of each unit writes the output.
-  a.unit_done = c->offloaded ? nullptr : c->unit_done;
-  a.done_ctr = (fold_advance && !c->offloaded) ? c->done_ctr : nullptr;
-  NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st));
+  a.unit_done = c->unit_done;
+  a.done_ctr = fold_advance ? c->done_ctr : nullptr;
   if (c->offloaded) {
-    // misses pass: one CTA per unit attends to the fetched blocks once the
-    // gather has landed and merges every partial of the unit into the output
-    if (c->gather_on_side) NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
-    a.unit_done = nullptr;
-    a.done_ctr = fold_advance ? c->done_ctr : nullptr;
-    NOSA_CUDA(launch_attend_misses(a, c->maps, st));
+    // the misses: copied from host memory into their cache slots and attended
+    // as they land, on the copy stream given to the fetch call, beside the
+    // hits pass
+    GatherAttendArgs ga{};
+    ga.g.hk = c->kv_k;
+    ga.g.hv = c->kv_v;
+    ga.g.ck = c->cache_k;
+    ga.g.cv = c->cache_v;
+    ga.g.glist = c->glist;
+    ga.g.count = &c->ds->gather_count;
+    ga.g.stage_k = c->stage_k;
+    ga.g.stage_v = c->stage_v;
+    ga.g.ds = c->ds;
+    ga.g.U = c->U;
+    ga.g.C = c->C;
+    ga.g.max_blocks = c->max_blocks;
+    ga.d = a;
+    if (c->gather_on_side) {
+      NOSA_CUDA(cudaEventRecord(c->ev_plan, st));
+      NOSA_CUDA(cudaStreamWaitEvent(c->copy_stream, c->ev_plan, 0));
+      NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, c->copy_stream));
+      NOSA_CUDA(cudaEventRecord(c->ev_gather, c->copy_stream));
+    } else {
+      NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, st));
+    }
   }
+  // hits pass: blocks already on the GPU (all of S(t) when KV is in HBM) plus
+  // the open tail
+  NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st));
+  if (c->gather_on_side) NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
   if (c->appends_enabled) {
     CloseArgs cl{};
     cl.tail_k = c->tail_k;

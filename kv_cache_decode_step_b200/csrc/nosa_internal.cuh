@@ -297,10 +297,11 @@ struct DecodeArgs {
   int resident;             // 1: sel indexes the resident KV
   int tail_split;           // 1: each unit's open tail is attended in the hits pass
   int part_base, nparts;    // hits pass writes slots part_base + segment; nparts per unit
+  int miss_base;            // slot of a unit's first fetched-block partial
   int hits_grid;            // CTAs of the hits pass (fixes each unit's segment count)
-  int* unit_done;           // resident: per-unit counters, the last CTA merges (else null)
+  int* unit_done;           // [U] partials written this step; completing one merges the unit
   uint16_t* out;            // [B, Hq, d]
-  int* done_ctr;            // non-null: the kernel's last CTA ends the step (advance_step)
+  int* done_ctr;            // non-null: units merged; the last merge ends the step (advance_step)
   DevStats* st;
 };
 struct DecodeMaps {
@@ -314,9 +315,27 @@ cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int gri
 int attend_hits_grid(int U, int k, int tail_split, int want);
 // Partial slots per unit the hits pass writes for this shape and requested grid.
 int attend_hits_parts(int U, int k, int tail_split, int want);
-// Misses pass: one CTA per unit, merges parts [0, part_base) into out.
-cudaError_t launch_attend_misses(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t st);
+// Kernel attributes (shared memory) of the attention kernels; once per device.
 cudaError_t configure_decode();
+cudaError_t configure_gather_attend();
+
+// The miss gather fused with the attention of each fetched block: copies every
+// entry of the gather list into its cache slot and, from shared memory, writes
+// the block's partial (slot miss_base + entry.w of its unit), merging the unit
+// when that completes its partials.  Highest CTA priority.
+struct GatherAttendArgs {
+  GatherArgs g;
+  DecodeArgs d;
+};
+cudaError_t launch_gather_attend(const GatherAttendArgs& a, int grid, cudaStream_t st);
+
+// Named barriers (bar.sync / bar.arrive over `count` threads, whole warps).
+__device__ __forceinline__ void bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 struct AppendArgs {
   const uint16_t* k_new;    // [B, Hkv, d]

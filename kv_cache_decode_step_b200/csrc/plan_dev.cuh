@@ -5,7 +5,8 @@
 // NOSA: Native and Offloadable Sparse Attention (paperlayer summary), §4 and
 // App. A.  Replacement order: free slots (lowest first), then resident blocks
 // outside S(t) by (last step selected, block id) ascending; the i-th miss
-// (ascending block id) takes the i-th slot of that order.
+// (ascending block id) takes the i-th slot of that order.  A gather-list
+// entry is (unit, block, slot, i): the block is the unit's i-th miss.
 #pragma once
 
 #include "nosa_internal.cuh"
@@ -126,7 +127,7 @@ __device__ __forceinline__ void plan_unit_smem(const PlanArgs& a, int u, int lan
       last_used[c] = t;
       items[n_hit + i] = c;
       fetch[i] = bj;
-      a.glist[base + i] = make_int4(u, bj, c, 0);
+      a.glist[base + i] = make_int4(u, bj, c, i);
     } else {
       fetch[i] = -1;
     }
@@ -227,7 +228,7 @@ __device__ __forceinline__ void plan_unit_reg(const PlanArgs& a, int u, int lane
     block_slot[bj] = c;
     items[n_hit + mi] = c;
     a.fetch[(size_t)u * a.k + mi] = bj;
-    a.glist[base + mi] = make_int4(u, bj, c, 0);
+    a.glist[base + mi] = make_int4(u, bj, c, mi);
   }
   for (int i = n_miss + lane; i < a.k; i += 32) a.fetch[(size_t)u * a.k + i] = -1;
   if (lane == 0) {
