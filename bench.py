@@ -363,6 +363,12 @@ def run_ours(args):
         dominant, other = rl_gather, None
     else:
         dominant, other = rl_attn, None
+    tr = NCU_TRAFFIC.get((dominant["kernel"], w.name))
+    if tr:
+        dominant["traffic"] = tr["dram"]
+        if "pcie_read" in tr:
+            dominant["traffic_pcie_read"] = tr["pcie_read"]
+        dominant["traffic_source"] = "ncu --set full capture of this kernel on this workload (bytes per launch)"
 
     result = None
     if rank == 0:
@@ -481,6 +487,14 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
 
 
 LATENCY_STEPS = 256
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu --set
+# full capture of the dominant kernel on its workload (pcie: link-level read
+# bytes, the traffic that bounds the gather).  Retake after changing the kernel.
+NCU_TRAFFIC = {
+    ("gather_attend_kernel", "offload_b64"): {"dram": 433152 + 12032, "pcie_read": 20715800},
+    ("attend_hits_kernel", "layer8b"): {"dram": 268967936 + 6740224},
+}
 
 
 def step_latency_pass(torch, dec, w, n):

@@ -297,8 +297,11 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   }
   if (const char* v = getenv("NOSA_GATHER_CTAS")) c->gather_grid = atoi(v) > 0 ? atoi(v) : c->gather_grid;
   // two persistent attention CTAs per SM, each over an equal share of the
-  // (unit, block) positions; a unit's blocks span a few CTAs' shares
-  int want = 2 * sms;
+  // (unit, block) positions; a unit's blocks span a few CTAs' shares.  With KV
+  // in host memory each gather CTA's shared memory leaves room for one
+  // attention CTA on its SM, so the grid shrinks to stay in one wave.
+  int want = 2 * sms - (c->offloaded ? c->gather_grid : 0);
+  if (want < sms) want = sms;
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
   c->attn_grid = attend_hits_grid(c->U, c->k, 1, want);
   c->hits_parts = attend_hits_parts(c->U, c->k, 1, c->attn_grid);
@@ -876,6 +879,7 @@ nosa_status nosa_set_state(nosa_ctx* c, const void* buf, size_t size) {
   d.staged_block = -1;
   d.wt_block = -1;
   d.wt_done = 0;
+  d.gather_next = 0;
   const size_t U = c->U, KE = c->cfg.k_agnostic > 0 ? c->cfg.k_agnostic : 1;
   auto put = [&](void* dev, size_t bytes) -> nosa_status {
     NOSA_CUDA(cudaMemcpy(dev, p, bytes, cudaMemcpyHostToDevice));

@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(PlanArgs a) {
   extern __shared__ int sm_plan[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * kPlanWarps + warp;
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.ds->gather_next = 0;  // see prepare_kernel
   if (u >= a.U) return;
   plan_unit_smem(a, u, lane, sm_plan + (size_t)warp * (2 * a.C + 2 * a.k), a.sel + (size_t)u * a.k,
                  a.block_slot + (size_t)u * a.max_blocks, false);
@@ -32,6 +33,7 @@ __global__ void __launch_bounds__(kPlanWarps * 32) plan_reg_kernel(PlanArgs a) {
   __shared__ int ssrc_all[kPlanWarps][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * kPlanWarps + warp;
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.ds->gather_next = 0;  // see prepare_kernel
   if (u >= a.U) return;
   plan_unit_reg(a, u, lane, ssrc_all[warp], a.sel + (size_t)u * a.k, a.slot_block + (size_t)u * a.C,
                 a.last_used + (size_t)u * a.C);

@@ -20,8 +20,8 @@
 // PCIe throughput follows the number of warps with loads in flight, hence the
 // larger copy role.
 // The roles hand stages over with named barriers (FULL: copy -> attention,
-// EMPTY: attention -> copy); both walk the same entries, so every barrier
-// phase has all its arrivals.  Nothing waits on another CTA or kernel.
+// EMPTY: attention -> copy), the entry riding with the stage, so every
+// barrier phase has all its arrivals.  Nothing waits on another CTA or kernel.
 #include "attend_dev.cuh"
 
 namespace nosa {
@@ -32,10 +32,11 @@ constexpr int kGaThreads = kGaCopy + kGaRole;
 constexpr int kGaStages = 2;
 constexpr int kGaStageBytes = 2 * kBlockBytes;
 constexpr int kGaWsBytes = (4 * kMaxG * kD + 2 * 4 * kMaxG) * 4;
-constexpr int kGaSmemBytes = kGaStages * kGaStageBytes + kGaWsBytes + 16;  // + flag, count, staged
+constexpr int kGaSmemBytes = kGaStages * kGaStageBytes + kGaWsBytes + 32;  // + flag, count, staged, 2 entries
 constexpr int kBarFull = 1;               // ids 1, 2: stage s full
 constexpr int kBarEmpty = 3;              // ids 3, 4: stage s free
 constexpr int kBarAttn = 5;               // the attention warps alone
+constexpr int kBarCopy = 6;               // the copy warps alone
 constexpr int kGaPer = kBlockBytes / 16 / kGaCopy;  // 16-byte words of K (and of V) per copy thread
 
 __device__ __forceinline__ uint4 ld_host(const uint4* p) {
@@ -44,6 +45,11 @@ __device__ __forceinline__ uint4 ld_host(const uint4* p) {
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;
+}
+
+__device__ __forceinline__ bool entry_valid(const GatherArgs& g, const DecodeArgs& a, const int4& it) {
+  return it.x >= 0 && it.x < g.U && it.y >= 0 && it.y < g.max_blocks && it.z >= 0 && it.z < g.C && it.w >= 0 &&
+         it.w < a.k;
 }
 
 __global__ void __launch_bounds__(kGaThreads, 1) gather_attend_kernel(GatherAttendArgs p) {
@@ -55,9 +61,9 @@ __global__ void __launch_bounds__(kGaThreads, 1) gather_attend_kernel(GatherAtte
   const int warp = rt >> 5, lane = threadIdx.x & 31;
   const WarpStates ws(ga_smem + kGaStages * kGaStageBytes);
   int* flag = reinterpret_cast<int*>(ga_smem + kGaStages * kGaStageBytes + kGaWsBytes);
-  // one read of the list length and of the staged block for the whole CTA,
-  // so that both roles walk the same entries (the last unit merged of the
-  // step clears the count)
+  // one read of the list length and of the staged block for the whole CTA
+  // (the last unit merged of the step clears the count)
+  int* s_entry = flag + 4;  // entry claimed for stage 0, 1
   if (threadIdx.x == 0) {
     flag[1] = *g.count;
     // the most recently closed block may not have reached the host store yet:
@@ -69,16 +75,25 @@ __global__ void __launch_bounds__(kGaThreads, 1) gather_attend_kernel(GatherAtte
   const int staged = flag[2];
   const auto attn_sync = [] { bar_sync(kBarAttn, kGaRole); };
 
-  int i = 0;
-  for (int e = blockIdx.x; e < count; e += gridDim.x, ++i) {
-    const int st = i & 1;
-    unsigned char* stage = ga_smem + st * kGaStageBytes;
-    const int4 it = g.glist[e];
-    const bool valid = it.x >= 0 && it.x < g.U && it.y >= 0 && it.y < g.max_blocks && it.z >= 0 && it.z < g.C &&
-                       it.w >= 0 && it.w < a.k;
-    if (!attn) {
+  // Entries are claimed one at a time from a device-wide counter, so CTAs
+  // that PCIe serves faster take more of them and all finish together.  The
+  // copy role claims and hands the entry to the attention role with the
+  // stage; a claim past the end is handed over as the signal to stop.
+  if (!attn) {
+    int i = 0;
+    for (;; ++i) {
+      const int st = i & 1;
+      unsigned char* stage = ga_smem + st * kGaStageBytes;
       if (i >= kGaStages) bar_sync(kBarEmpty + st, kGaThreads);
-      if (valid) {
+      if (rt == 0) s_entry[st] = atomicAdd(&g.ds->gather_next, 1);
+      bar_sync(kBarCopy, kGaCopy);
+      const int e = s_entry[st];
+      if (e >= count) {
+        bar_arrive(kBarFull + st, kGaThreads);
+        break;
+      }
+      const int4 it = g.glist[e];
+      if (entry_valid(g, a, it)) {
         const bool from_stage = it.y == staged;
         const size_t src = from_stage ? (size_t)it.x * (kBlockBytes / 16)
                                       : ((size_t)it.x * g.max_blocks + it.y) * (kBlockBytes / 16);
@@ -106,8 +121,19 @@ __global__ void __launch_bounds__(kGaThreads, 1) gather_attend_kernel(GatherAtte
         atomicOr(&g.ds->error_bits, ERR_RANGE);
       }
       bar_arrive(kBarFull + st, kGaThreads);
-    } else {
+    }
+    // i entries were real; take the EMPTY arrival of the last one, the only
+    // one not consumed inside the loop
+    if (i >= 1) bar_sync(kBarEmpty + ((i - 1) & 1), kGaThreads);
+  } else {
+    for (int i = 0;; ++i) {
+      const int st = i & 1;
+      unsigned char* stage = ga_smem + st * kGaStageBytes;
       bar_sync(kBarFull + st, kGaThreads);
+      const int e = s_entry[st];
+      if (e >= count) break;
+      const int4 it = g.glist[e];
+      const bool valid = entry_valid(g, a, it);
       AttnAcc acc;
       acc_init(acc);
       if (valid) {
@@ -116,7 +142,7 @@ __global__ void __launch_bounds__(kGaThreads, 1) gather_attend_kernel(GatherAtte
         const uint32_t kb = smem_u32(stage);
         attend_block(kb, kb + kBlockBytes, warp, lane, kP, qf, acc);
       }
-      bar_arrive(kBarEmpty + st, kGaThreads);  // the stage is read out
+      bar_arrive(kBarEmpty + st, kGaThreads);  // the stage (and its entry slot) is read out
       if (valid) {
         const int u = it.x;
         const size_t part = (size_t)u * a.nparts + a.miss_base + it.w;
@@ -126,9 +152,6 @@ __global__ void __launch_bounds__(kGaThreads, 1) gather_attend_kernel(GatherAtte
       }
     }
   }
-  // the copy warps take the EMPTY arrivals of the last stages they did not wait for
-  if (!attn)
-    for (int j = i > kGaStages ? i - kGaStages : 0; j < i; ++j) bar_sync(kBarEmpty + (j & 1), kGaThreads);
 }
 
 cudaError_t configure_gather_attend() {

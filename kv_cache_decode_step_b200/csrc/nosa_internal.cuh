@@ -37,7 +37,8 @@ struct DevState {
   int staged_block;    // closed block whose K/V sit in the staging buffer, -1 none
   int wt_block;        // staged block not yet written through to the store, -1 none
   int wt_done;         // CTAs of the write-through launch that have finished
-  int pad[2];
+  int gather_next;     // next gather-list entry to claim (reset by the kernel that plans the step)
+  int pad;
 };
 
 struct DevStats {

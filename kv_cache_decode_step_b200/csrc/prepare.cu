@@ -39,6 +39,9 @@ __global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs
   int* s_bs = s_lu + 32;  // general plan: the unit's block -> slot table [max_blocks]
   const int u = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the gather that follows claims its entries from 0 (it is the only user
+  // of this counter and runs after this kernel has completed)
+  if (u == 0 && threadIdx.x == 0) a.sc.ds->gather_next = 0;
   const bool reg_plan = a.offloaded && C <= 32 && k <= 32;
 
   // asynchronous copies: they land while the scores stream in

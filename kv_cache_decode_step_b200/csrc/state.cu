@@ -170,7 +170,8 @@ __global__ void init_state_kernel(DevState* ds, int n_closed, int tail_len, int 
   ds->staged_block = -1;
   ds->wt_block = -1;
   ds->wt_done = 0;
-  ds->pad[0] = ds->pad[1] = 0;
+  ds->gather_next = 0;
+  ds->pad = 0;
 }
 
 cudaError_t launch_init_state(DevState* ds, int n_closed, int tail_len, int step, int n_last_select,
