@@ -18,14 +18,15 @@
 //   Gamma_q(t) = top-k_q by score of (S(t-1) \ (F ∪ Gamma_e)) ∪ top-c_t(new)
 //   S(t)       = F(t) ∪ Gamma_e(t) ∪ Gamma_q(t), ties to the lower block id.
 //
-// Lane l owns the blocks j with j % 32 == l.  Up to 1024 blocks their keys sit
-// in registers and sets are per-lane bit masks; beyond that sets are bitmaps
-// in shared memory (bit l of word j / 32) and keys are read from memory.
-// Keys are order-preserving integer images of the
-// scores (larger score -> larger key), so one warp-wide argmax is two
-// redux.sync max steps, a ballot and, only on an exact tie, a redux.sync min
-// over block ids.  Choosing c of a set of p candidates takes min(c, p - c)
-// rounds: either move the c best out, or remove the p - c worst.
+// Lane l owns the blocks j with j % 32 == l.  Keys are order-preserving
+// integer images of the scores (larger score -> larger key).  Up to 1024
+// blocks the keys sit in registers and sets are per-lane bit masks, and a
+// top-c set is found by a bitwise search over the keys (select_dev.cuh).
+// Beyond that sets are bitmaps in shared memory (bit l of word j / 32), keys
+// are read from memory, and one warp-wide argmax -- two redux.sync max steps,
+// a ballot and, only on an exact tie, a redux.sync min over block ids --
+// moves one block per round: choosing c of p candidates takes min(c, p - c)
+// rounds, either moving the c best out or removing the p - c worst.
 #include <climits>
 
 #include "select_dev.cuh"

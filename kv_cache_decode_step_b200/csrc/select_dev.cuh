@@ -24,63 +24,67 @@ __device__ __forceinline__ unsigned long long key_f32(float x) {
 
 // ---------------------------------------------------------------- register path
 // For n <= 32 * R: lane l holds blocks j = 32 i + l (i < R) -- their keys in
-// registers and set membership as R-bit masks -- so a round of selection is a
-// warp_winner plus an R-step rescan in registers, and lists come out of one
-// ballot per row i.
+// registers and set membership as R-bit masks -- so choosing a top-c set is a
+// bitwise search with one warp-wide count per key bit, and lists come out of
+// one ballot per row i.
 
+// Keep exactly the c best of `mask` (per-lane R-bit masks, whole warp): the
+// c largest keys, the lower block id first among equal keys.  Radix
+// selection: the threshold key is fixed one bit at a time, most significant
+// first; `cand` holds the members that still agree with the threshold's
+// prefix, `kept` those already above it.  Each bit costs one warp-wide count
+// (redux.sync), and the search stops as soon as the candidates left are
+// exactly the ones still needed.  Members whose whole key equals the
+// threshold are then told apart the same way on their block ids
+// j = 32 i + lane (smaller ids first).
 template <int R>
-__device__ __forceinline__ void lane_best_reg(uint32_t mask, const unsigned long long (&k)[R], bool worst,
-                                              unsigned long long& bk, int& bi) {
-  bk = 0ull;
-  bi = -1;
+__device__ __forceinline__ void keep_best_reg(uint32_t& mask, int c, const unsigned long long (&k)[R], int lane) {
+  int left = (int)__reduce_add_sync(kFull, (unsigned)__popc(mask));  // members in cand
+  if (left <= c) return;
+  uint32_t kept = 0u, cand = mask;
+  int need = c;
+  // 64 key bits: the high words, then the low words
+#pragma unroll 1
+  for (int b = 63; b >= 0 && need > 0 && need < left; --b) {
+    uint32_t ones = 0u;
 #pragma unroll
-  for (int i = 0; i < R; ++i) {
-    if ((mask >> i) & 1u) {
-      const unsigned long long kk = worst ? ~k[i] : k[i];
-      // rows ascend with i: on equal keys keep the first for "best", the last for "worst"
-      if (bi < 0 || kk > bk || (worst && kk == bk)) {
-        bk = kk;
-        bi = i;
-      }
+    for (int i = 0; i < R; ++i) ones |= (uint32_t)((k[i] >> b) & 1ull) << i;
+    ones &= cand;
+    const int n1 = (int)__reduce_add_sync(kFull, (unsigned)__popc(ones));
+    if (n1 >= need) {  // the threshold has this bit set: members without it fall out
+      cand = ones;
+      left = n1;
+    } else {           // it has this bit clear: members with it are above the threshold
+      kept |= ones;
+      need -= n1;
+      cand &= ~ones;
+      left -= n1;
     }
   }
-}
-
-// Keep exactly the c best of `mask` (per-lane R-bit masks, whole warp).
-template <int R>
-__device__ void keep_best_reg(uint32_t& mask, int c, const unsigned long long (&k)[R], int lane) {
-  const int p = (int)__reduce_add_sync(kFull, (unsigned)__popc(mask));
-  if (p <= c) return;
-  const bool worst = (p - c) < c;
-  const int rounds = worst ? p - c : c;
-  uint32_t kept = 0u;
-  unsigned long long bk;
-  int bi;
-  lane_best_reg<R>(mask, k, worst, bk, bi);
-  for (int r = 0; r < rounds; ++r) {
-    const unsigned hi = (unsigned)(bk >> 32);
-    const unsigned mhi = __reduce_max_sync(kFull, hi);
-    if (mhi == 0u) break;
-    const unsigned lo = (bi >= 0 && hi == mhi) ? (unsigned)bk : 0u;
-    const unsigned mlo = __reduce_max_sync(kFull, lo);
-    const unsigned cand = __ballot_sync(kFull, bi >= 0 && hi == mhi && (unsigned)bk == mlo);
-    int wl;  // winning lane
-    if (__popc(cand) == 1) {
-      wl = __ffs(cand) - 1;
+  // equal keys: the smaller block ids (bits 5.. of j are the row i, bits 0..4 the lane)
+#pragma unroll 1
+  for (int b = 9; b >= 0 && need > 0 && need < left; --b) {
+    uint32_t zeros = 0u;
+    if (b >= 5) {
+#pragma unroll
+      for (int i = 0; i < R; ++i) zeros |= (((i >> (b - 5)) & 1) ? 0u : 1u) << i;
     } else {
-      // equal keys: block id 32*bi + lane decides (smaller for best, larger for worst)
-      const unsigned j = (unsigned)(32 * bi + lane);
-      const unsigned t = ((cand >> lane) & 1u) ? (worst ? ~j : j) : 0xffffffffu;
-      const unsigned mt = __reduce_min_sync(kFull, t);
-      wl = __ffs(__ballot_sync(kFull, ((cand >> lane) & 1u) && t == mt)) - 1;
+      zeros = ((lane >> b) & 1) ? 0u : 0xffffffffu;
     }
-    if (lane == wl) {
-      mask &= ~(1u << bi);
-      if (!worst) kept |= 1u << bi;
-      lane_best_reg<R>(mask, k, worst, bk, bi);
+    zeros &= cand;
+    const int n0 = (int)__reduce_add_sync(kFull, (unsigned)__popc(zeros));
+    if (n0 >= need) {
+      cand = zeros;
+      left = n0;
+    } else {
+      kept |= zeros;
+      need -= n0;
+      cand &= ~zeros;
+      left -= n0;
     }
   }
-  if (!worst) mask = kept;
+  if (need > 0) kept |= cand;  // need == left: every candidate left is in
+  mask = kept;
 }
 
 // Blocks of the per-lane masks, ascending, into out[0..cap); returns the count.
@@ -88,7 +92,7 @@ template <int R>
 __device__ __forceinline__ int write_list_reg(uint32_t mask, int* out, int cap, int lane) {
   const unsigned lt = (1u << lane) - 1u;
   int base = 0;
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < R; ++i) {
     const bool on = (mask >> i) & 1u;
     const unsigned bal = __ballot_sync(kFull, on);
