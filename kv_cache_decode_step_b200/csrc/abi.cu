@@ -132,6 +132,7 @@ struct nosa_ctx {
   bool wt_forked = false;
   int wt_grid = 18;
   int prep_warps = 4;       // warps per CTA of the fused score/select/plan kernel
+  int attn_stages = 3;      // TMA stages per hits-pass CTA
 };
 
 namespace {
@@ -302,6 +303,8 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   // attention CTA on its SM, so the grid shrinks to stay in one wave.
   int want = 2 * sms - (c->offloaded ? c->gather_grid : 0);
   if (want < sms) want = sms;
+  if (const char* v = getenv("NOSA_ATTN_STAGES")) c->attn_stages = atoi(v) == 2 ? 2 : 3;
+  if (c->attn_stages == 2) want = 3 * sms - (c->offloaded ? c->gather_grid : 0);
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
   c->attn_grid = attend_hits_grid(c->U, c->k, 1, want);
   c->hits_parts = attend_hits_parts(c->U, c->k, 1, c->attn_grid);
@@ -707,7 +710,7 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
   }
   // hits pass: blocks already on the GPU (all of S(t) when KV is in HBM) plus
   // the open tail
-  NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st));
+  NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st, c->attn_stages));
   if (c->gather_on_side) NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
   if (c->appends_enabled) {
     CloseArgs cl{};

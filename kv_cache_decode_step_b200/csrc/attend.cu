@@ -19,12 +19,11 @@
 
 namespace nosa {
 
-constexpr int kStages = 3;
 constexpr int kAttnThreads = 128;
 constexpr int kStageBytes = 2 * kBlockBytes;
-constexpr int kBarOffset = kStages * kStageBytes;
-constexpr int kFlagOffset = kBarOffset + kStages * 8;
-constexpr int kSmemBytes = kFlagOffset + 16 + 1024;  // + slack for 1024-byte alignment
+// Shared memory of a CTA with S stages: the stages, S mbarriers, a flag word
+// and slack for 1024-byte alignment.
+constexpr int smem_bytes_for(int S) { return S * kStageBytes + S * 8 + 16 + 1024; }
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 // Issue the TMA loads of one block (K and V: four 64 x 64 boxes, 32 KiB).
@@ -66,12 +65,13 @@ __device__ __forceinline__ bool position_valid(const DecodeArgs& a, int j, int n
   return tail_len > 0;
 }
 
+template <int kStages>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attend_hits_kernel(const __grid_constant__ DecodeMaps maps, DecodeArgs a) {
   extern __shared__ unsigned char attn_smem_raw[];
   unsigned char* sm = aligned_smem(attn_smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kBarOffset);
-  int* s_flag = reinterpret_cast<int*>(sm + kFlagOffset);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kStages * kStageBytes);
+  int* s_flag = reinterpret_cast<int*>(sm + kStages * kStageBytes + kStages * 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tail_len = a.tail_split ? a.ds->tail_len_step : 0;
   Walk wk;
@@ -179,17 +179,25 @@ __host__ __device__ inline int hits_segments_per_unit(int U, int vpu, int grid) 
   return (int)(((long long)vpu * grid + V - 1) / V) + 1;
 }
 
-int attend_smem_bytes() { return kSmemBytes; }
+int attend_smem_bytes() { return smem_bytes_for(3); }
 
 // Called once per context creation (on its device), outside any stream capture.
 cudaError_t configure_decode() {
-  cudaError_t e = cudaFuncSetAttribute(attend_hits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(attend_hits_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem_bytes_for(3));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attend_hits_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes_for(2));
   if (e != cudaSuccess) return e;
   return configure_gather_attend();
 }
 
-cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st) {
-  attend_hits_kernel<<<grid, kAttnThreads, kSmemBytes, st>>>(m, a);
+// stages: TMA stages per CTA (2 or 3); the grid's CTAs per SM follow from it.
+cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st, int stages) {
+  if (stages == 2) {
+    attend_hits_kernel<2><<<grid, kAttnThreads, smem_bytes_for(2), st>>>(m, a);
+  } else {
+    attend_hits_kernel<3><<<grid, kAttnThreads, smem_bytes_for(3), st>>>(m, a);
+  }
   return cudaGetLastError();
 }
 

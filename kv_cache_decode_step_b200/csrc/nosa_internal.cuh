@@ -311,7 +311,8 @@ struct DecodeMaps {
 };
 // Hits pass (persistent, `grid` CTAs, which must equal a.hits_grid); partials,
 // and with unit_done the output.
-cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st);
+cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st,
+                               int stages = 3);
 // The hits-pass grid for a requested CTA count (at most one CTA per position).
 int attend_hits_grid(int U, int k, int tail_split, int want);
 // Partial slots per unit the hits pass writes for this shape and requested grid.
