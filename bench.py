@@ -479,8 +479,8 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
     out["fetched_bytes_per_step"] = (dec.stats()["fetched_bytes"] - fb0) / n
     out["steps"] = n
     out["single_stream"] = bool(single_stream)
-    out["fused_prepare"] = bool(dec.fused)
-    if dec.fused:
+    out["fused_prepare"] = bool(dec.fused and w.max_blocks <= 512)
+    if out["fused_prepare"]:
         for k in ("score_ms", "select_ms", "plan_ms"):
             out.pop(k)
     return out
