@@ -143,3 +143,14 @@ def test_fused_and_separate_calls_agree_bit_exactly(name, kw, graph):
         for x, y in zip(a.resident[t], b.resident[t]):
             assert np.array_equal(x, y)
     assert a.stats == b.stats
+
+
+@pytest.mark.parametrize("offloaded", [True, False])
+def test_two_stage_hits_pass(offloaded, monkeypatch):
+    """The hits pass built with two TMA stages (three CTAs per SM), chosen
+    by NOSA_ATTN_STAGES=2 when the context is created."""
+    monkeypatch.setenv("NOSA_ATTN_STAGES", "2")
+    w = configs.get("layer8b", batch=2, steps=12)
+    if offloaded:
+        w = w.with_(offloaded=True, cache_factor=2)
+    _full(w, range(w.units), range(w.steps), cache_steps=[w.steps - 1] if offloaded else ())
