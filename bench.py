@@ -334,8 +334,9 @@ def run_ours(args):
     latency = step_latency_pass(torch, dec, w, LATENCY_STEPS)
 
     # ---- end to end through host buffers: q from pinned host, out to pinned host
-    e2e = e2e_pass(torch, dec, w, nosa, args.e2e_steps)
-    e2e["eager_value"] = e2e_pass(torch, dec, w, nosa, args.e2e_steps, eager=True)["value"]
+    e2e = e2e_pass(torch, dec, w, nosa, args.e2e_steps, dist=dist, world=world, dev=dev)
+    e2e["eager_value"] = e2e_pass(torch, dec, w, nosa, args.e2e_steps, eager=True, dist=dist, world=world,
+                                  dev=dev)["value"]
 
     # kernels per step: score, select, [plan, gather + miss attention], hits
     # pass -- the fused entry point makes score, select and plan one kernel up
@@ -523,7 +524,7 @@ def step_latency_pass(torch, dec, w, n):
     return out
 
 
-def e2e_pass(torch, dec, w, nosa, n, eager=False):
+def e2e_pass(torch, dec, w, nosa, n, eager=False, dist=None, world=1, dev=None):
     """End to end through the binding, as a decode loop would run it: every
     step copies that step's inputs (q, and for growing sequences the new
     token's K/V) from pinned host memory, replays the captured step and reads
@@ -537,6 +538,8 @@ def e2e_pass(torch, dec, w, nosa, n, eager=False):
     s = dec.stream
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     e0.record(s)
     t0 = time.perf_counter()
     for _ in range(n):
@@ -555,11 +558,13 @@ def e2e_pass(torch, dec, w, nosa, n, eager=False):
     e1.record(s)
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
-    ms = e0.elapsed_time(e1)
+    # whole job: every rank decodes its own batch; the slowest rank's time
+    ms = max_over_ranks(torch, dist, e0.elapsed_time(e1), dev, world)
+    wall = max_over_ranks(torch, dist, wall * 1e3, dev, world) * 1e-3
     qb = dec.q.numel() * 2 + sum(d.numel() * d.element_size() for d, _ in extra)
     ob = dec.out.numel() * 2
-    return {"value": w.batch * n / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": qb,
-            "d2h_bytes_per_step": ob, "steps": n, "wall_tokens_per_s": w.batch * n / wall,
+    return {"value": world * w.batch * n / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": qb,
+            "d2h_bytes_per_step": ob, "steps": n, "wall_tokens_per_s": world * w.batch * n / wall,
             "note": "captured step replayed through the binding; inputs H2D from pinned host and the output "
                     "D2H inside the timed region, host waits for each step's output"}
 

@@ -154,3 +154,18 @@ def test_two_stage_hits_pass(offloaded, monkeypatch):
     if offloaded:
         w = w.with_(offloaded=True, cache_factor=2)
     _full(w, range(w.units), range(w.steps), cache_steps=[w.steps - 1] if offloaded else ())
+
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_cache_of_exactly_k_slots(graph):
+    """C = k: a full cache holds exactly S(t-1), so every miss evicts a block
+    the step does not use; queries resampled every 4 steps force many misses."""
+    w = configs.get("tiny", cache_factor=1, steps=24, resample_every=4)
+    data = inputs.generate(w)
+    sample = list(range(w.units))
+    attend = list(range(w.steps))
+    rec = run_gpu(w, data, sample, attend, graph=graph, cache_steps=[3, 4, 12, w.steps - 1])
+    refs = run_oracle(w, data, sample, attend)
+    compare(w, rec, refs, sample)
+    check_all_unit_invariants(w, rec, w.steps)
+    assert rec.stats["misses"] > w.units * w.steps  # the resamples made it miss
