@@ -76,7 +76,11 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # the raw samples (NOSA_CLOCKS_DIR, default the temp directory); the
+        # bench line carries their summary
+        import tempfile
+        d = os.environ.get("NOSA_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(d, f"nosa_clocks_gpu{gpu_index}.csv")
         self.t0 = self.t1 = None
 
     def start(self):
