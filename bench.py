@@ -73,14 +73,14 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
         self.proc = None
         # the raw samples (NOSA_CLOCKS_DIR, default the temp directory); the
         # bench line carries their summary
         import tempfile
         d = os.environ.get("NOSA_CLOCKS_DIR") or tempfile.gettempdir()
-        self.path = os.path.join(d, f"nosa_clocks_gpu{gpu_index}.csv")
+        self.path = os.path.join(d, "nosa_clocks_%s.csv" % gpu_id.replace(":", "_").replace(".", "_"))
         self.t0 = self.t1 = None
 
     def start(self):
@@ -146,6 +146,37 @@ def max_over_ranks(torch, dist, ms_local, device, world):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def gpu_pci_bus_id(torch, local):
+    """PCI bus id of CUDA device `local` (NVML and nvidia-smi number devices
+    differently once CUDA_VISIBLE_DEVICES is set)."""
+    pr = torch.cuda.get_device_properties(local)
+    return f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+
+
+def bind_to_gpu_numa_node(bus_id):
+    """Restrict this process to the CPUs nearest the GPU before any pinned
+    allocation, so that pinned host memory (the offloaded KV the gather reads
+    over PCIe) is allocated on the GPU's NUMA node.  Reads the affinity from
+    NVML; changes no GPU setting.  Returns the CPU count, or None."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus_id)
+            ncpu = os.cpu_count() or 1
+            words = pynvml.nvmlDeviceGetCpuAffinity(h, (ncpu + 63) // 64)
+        finally:
+            pynvml.nvmlShutdown()
+        cpus = {64 * i + b for i, wd in enumerate(words) for b in range(64) if (int(wd) >> b) & 1}
+        cpus &= os.sched_getaffinity(0)
+        if not cpus:
+            return None
+        os.sched_setaffinity(0, cpus)
+        return len(cpus)
+    except Exception:
+        return None
 
 
 def job_tokens_per_s(world, batch, steps, ms_max):
@@ -265,6 +296,8 @@ def run_ours(args):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    bus_id = gpu_pci_bus_id(torch, local)
+    numa_cpus = bind_to_gpu_numa_node(bus_id)
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
@@ -288,7 +321,7 @@ def run_ours(args):
     nosa.nosa_reset_stats(dec.ctx, dec.stream)
 
     # ---- timed region: K graph replays
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(bus_id)
     clocks.start()
     time.sleep(1.0)  # let the sampler start before the timed window
     if world > 1:
@@ -395,6 +428,7 @@ def run_ours(args):
                        "l2": (f"per-step HBM traffic {hbm_bytes / 2**20:.0f} MiB "
                               + ("> 126 MB L2, no flush" if hbm_bytes > 126e6 else "< 126 MB L2, not flushed")),
                        "graph": "cuda graph replay",
+                       "cpu_affinity": (f"{numa_cpus} CPUs local to the GPU" if numa_cpus else "unchanged"),
                        "calls": ("nosa_score_select_fetch (fused) + nosa_sparse_decode" if fused
                                  else "nosa_score_blocks + nosa_select + nosa_fetch_missing + nosa_sparse_decode")},
             "roofline": dominant,
