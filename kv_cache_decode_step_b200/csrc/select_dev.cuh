@@ -87,17 +87,24 @@ __device__ __forceinline__ void keep_best_reg(uint32_t& mask, int c, const unsig
   mask = kept;
 }
 
-// Blocks of the per-lane masks, ascending, into out[0..cap); returns the count.
+// Blocks of the per-lane masks, ascending, into out[0..cap) and, when given,
+// into out2 and out3 as well (one walk over the rows); returns the count.
 template <int R>
-__device__ __forceinline__ int write_list_reg(uint32_t mask, int* out, int cap, int lane) {
+__device__ __forceinline__ int write_list_reg(uint32_t mask, int* out, int cap, int lane, int* out2 = nullptr,
+                                              int* out3 = nullptr) {
   const unsigned lt = (1u << lane) - 1u;
   int base = 0;
-#pragma unroll 1
+#pragma unroll 4
   for (int i = 0; i < R; ++i) {
     const bool on = (mask >> i) & 1u;
     const unsigned bal = __ballot_sync(kFull, on);
     const int pos = base + __popc(bal & lt);
-    if (on && pos < cap) out[pos] = 32 * i + lane;
+    if (on && pos < cap) {
+      const int j = 32 * i + lane;
+      out[pos] = j;
+      if (out2) out2[pos] = j;
+      if (out3) out3[pos] = j;
+    }
     base += __popc(bal);
   }
   return base;
@@ -184,9 +191,7 @@ __device__ __forceinline__ void select_unit_reg(const SelectArgs& a, int u, int 
   const int ov = (int)__reduce_add_sync(kFull, (unsigned)__popc(mS & mP));
 
   int* sel = a.sel + (size_t)u * a.k;
-  const int ns = write_list_reg<R>(mS, sel, a.k, lane);
-  write_list_reg<R>(mS, prev, a.k, lane);
-  if (sel_copy) write_list_reg<R>(mS, sel_copy, a.k, lane);
+  const int ns = write_list_reg<R>(mS, sel, a.k, lane, prev, sel_copy);
   for (int i = ns + lane; i < a.k; i += 32) {
     sel[i] = -1;
     prev[i] = -1;
