@@ -81,6 +81,7 @@ __device__ __forceinline__ void plan_unit_smem(const PlanArgs& a, int u, int lan
   bool failed = false;
   while (n_src < n_miss) {
     unsigned bhi = 0xffffffffu, blo = 0xffffffffu;
+    int bc = -1;  // this lane's best candidate slot
     for (int c = lane; c < a.C; c += 32) {
       const int bj = sb[c];
       const int st = lu[c];
@@ -89,6 +90,7 @@ __device__ __forceinline__ void plan_unit_smem(const PlanArgs& a, int u, int lan
         if (h < bhi || (h == bhi && l < blo)) {
           bhi = h;
           blo = l;
+          bc = c;
         }
       }
     }
@@ -98,11 +100,12 @@ __device__ __forceinline__ void plan_unit_smem(const PlanArgs& a, int u, int lan
       failed = true;
       break;
     }
+    // slots hold distinct blocks: exactly one lane holds the winner's slot
+    const unsigned win = __ballot_sync(kAll, bc >= 0 && bhi == mhi && blo == mlo);
+    const int vslot = __shfl_sync(kAll, bc, __ffs(win) - 1);
     if (lane == 0) {
-      const int victim_block = (int)mlo;
-      const int vslot = bs_in[victim_block];  // a victim is not selected: its entry is unchanged
       ssrc[n_src] = vslot;
-      block_slot[victim_block] = -1;
+      block_slot[mlo] = -1;
       sb[vslot] = -2;  // claimed; excluded from the search
       lu[vslot] = t;
     }
