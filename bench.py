@@ -531,8 +531,8 @@ LATENCY_STEPS = 256
 # full capture of the dominant kernel on its workload (pcie: link-level read
 # bytes, the traffic that bounds the gather).  Retake after changing the kernel.
 NCU_TRAFFIC = {
-    ("gather_attend_kernel", "offload_b64"): {"dram": 433152 + 12032, "pcie_read": 20715800},
-    ("attend_hits_kernel", "layer8b"): {"dram": 268967936 + 6740224},
+    ("gather_attend_kernel", "offload_b64"): {"dram": 453632 + 14080, "pcie_read": 20715513},
+    ("attend_hits_kernel", "layer8b"): {"dram": 268933376 + 4087040},
 }
 
 
