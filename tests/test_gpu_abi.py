@@ -43,6 +43,37 @@ def test_step_calls_out_of_order_are_rejected(tiny):
         dec.close()
 
 
+def test_fused_first_half_follows_the_same_order(tiny):
+    """nosa_score_select_fetch stands for score + select + fetch: it starts a
+    step, cannot be repeated, and is followed by the decode call only."""
+    w, data = tiny
+    dec = runner.Decoder(w, data)
+    try:
+        s = dec.stream
+        args = (dec.ctx, dec.q, dec.scores, dec.sel, dec.fetch, dec.n_fetch, s, s)
+        nosa.nosa_score_blocks(dec.ctx, dec.q, dec.scores, s)
+        with pytest.raises(nosa.NosaError) as e:  # a step is already under way
+            nosa.nosa_score_select_fetch(*args)
+        assert e.value.status == nosa.NOSA_ERR_ORDER
+        nosa.nosa_select(dec.ctx, dec.scores, dec.sel, s)
+        nosa.nosa_fetch_missing(dec.ctx, dec.sel, dec.fetch, dec.n_fetch, s, s)
+        nosa.nosa_sparse_decode(dec.ctx, dec.q, dec.sel, dec.out, s)
+        nosa.nosa_score_select_fetch(*args)
+        with pytest.raises(nosa.NosaError) as e:
+            nosa.nosa_score_select_fetch(*args)
+        assert e.value.status == nosa.NOSA_ERR_ORDER
+        with pytest.raises(nosa.NosaError) as e:
+            nosa.nosa_select(dec.ctx, dec.scores, dec.sel, s)
+        assert e.value.status == nosa.NOSA_ERR_ORDER
+        nosa.nosa_sparse_decode(dec.ctx, dec.q, dec.sel, dec.out, s)
+        with pytest.raises(nosa.NosaError) as e:  # NULL outputs are rejected before any launch
+            nosa.nosa_score_select_fetch(dec.ctx, dec.q, dec.scores, dec.sel, None, dec.n_fetch, s, s)
+        assert e.value.status == nosa.NOSA_ERR_INVALID
+        dec.check()
+    finally:
+        dec.close()
+
+
 def test_pointer_kinds_are_checked(tiny):
     w, data = tiny
     ctx = nosa.nosa_create(nosa.config_from_workload(w))
