@@ -179,8 +179,6 @@ __host__ __device__ inline int hits_segments_per_unit(int U, int vpu, int grid) 
   return (int)(((long long)vpu * grid + V - 1) / V) + 1;
 }
 
-int attend_smem_bytes() { return smem_bytes_for(3); }
-
 // Called once per context creation (on its device), outside any stream capture.
 cudaError_t configure_decode() {
   cudaError_t e = cudaFuncSetAttribute(attend_hits_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
