@@ -57,6 +57,7 @@ def _cfg(**kw):
     ("n_q_heads", 36, nosa.NOSA_ERR_UNIMPLEMENTED),   # group of 18 > 8
     ("batch", 0, nosa.NOSA_ERR_INVALID),
     ("k_query", -1, nosa.NOSA_ERR_INVALID),
+    ("k_query", 253, nosa.NOSA_ERR_UNIMPLEMENTED),    # k = 257 > 256
     ("min_overlap", 17, nosa.NOSA_ERR_INVALID),       # > k = 16
     ("min_overlap", -1, nosa.NOSA_ERR_INVALID),
     ("max_blocks", 15, nosa.NOSA_ERR_INVALID),        # < k
