@@ -406,7 +406,7 @@ def run_ours(args):
         dominant["traffic"] = tr["dram"]
         if "pcie_read" in tr:
             dominant["traffic_pcie_read"] = tr["pcie_read"]
-        dominant["traffic_source"] = "ncu --set full capture of this kernel on this workload (bytes per launch)"
+        dominant["traffic_source"] = "ncu capture of this kernel on this workload (bytes per launch)"
 
     result = None
     if rank == 0:
@@ -531,8 +531,7 @@ LATENCY_STEPS = 256
 # full capture of the dominant kernel on its workload (pcie: link-level read
 # bytes, the traffic that bounds the gather).  Retake after changing the kernel.
 NCU_TRAFFIC = {
-    ("gather_attend_kernel", "offload_b64"): {"dram": 453632 + 14080, "pcie_read": 20715513},
-    ("attend_hits_kernel", "layer8b"): {"dram": 268933376 + 4087040},
+    ("gather_attend_kernel", "offload_b64"): {"dram": 590848 + 29440, "pcie_read": 20717568},
 }
 
 

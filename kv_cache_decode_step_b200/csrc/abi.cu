@@ -118,7 +118,7 @@ struct nosa_ctx {
   bool h_appended = false, appends_enabled = false;
   Phase phase = kReady;
 
-  int nparts = 2, hits_parts = 2, gather_grid = 148, attn_grid = 296;
+  int nparts = 2, hits_parts = 2, gather_grid = 148, attn_grid = 296, hits_vpu = 1;
   int* unit_done = nullptr;
   int* done_ctr = nullptr;
 
@@ -306,8 +306,12 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   if (const char* v = getenv("NOSA_ATTN_STAGES")) c->attn_stages = atoi(v) == 2 ? 2 : 3;
   if (c->attn_stages == 2) want = 3 * sms - (c->offloaded ? c->gather_grid : 0);
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
-  c->attn_grid = attend_hits_grid(c->U, c->k, 1, want);
-  c->hits_parts = attend_hits_parts(c->U, c->k, 1, c->attn_grid);
+  // the hits pass walks k blocks, the open tail and kHitsGap empty positions per unit
+  int gap = kHitsGap;
+  if (const char* v = getenv("NOSA_ATTN_GAP")) gap = atoi(v) >= 0 && atoi(v) <= 64 ? atoi(v) : gap;
+  c->hits_vpu = c->k + 1 + gap;
+  c->attn_grid = attend_hits_grid(c->U, c->hits_vpu, want);
+  c->hits_parts = attend_hits_parts(c->U, c->hits_vpu, c->attn_grid);
   // partial slots per unit: the hits pass's segments, then one per fetched block
   c->nparts = c->hits_parts + (c->offloaded ? c->k : 0);
 
@@ -669,6 +673,7 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
   a.C = c->C;
   a.resident = c->offloaded ? 0 : 1;
   a.tail_split = 1;
+  a.vpu = c->hits_vpu;
   a.nparts = c->nparts;
   a.part_base = 0;
   a.hits_grid = c->attn_grid;

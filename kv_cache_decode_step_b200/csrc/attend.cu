@@ -62,7 +62,7 @@ __device__ __forceinline__ void issue_block(const DecodeMaps& m, const DecodeArg
 
 __device__ __forceinline__ bool position_valid(const DecodeArgs& a, int j, int n_hit_u, int tail_len) {
   if (j < a.k) return a.resident ? true : j < n_hit_u;
-  return tail_len > 0;
+  return j == a.k && tail_len > 0;  // the open tail; positions past it are the unit's gap
 }
 
 template <int kStages>
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tail_len = a.tail_split ? a.ds->tail_len_step : 0;
   Walk wk;
-  wk.vpu = a.k + a.tail_split;
+  wk.vpu = a.vpu;
   wk.V = (long long)a.U * wk.vpu;
   wk.grid = gridDim.x;
   const long long p0 = wk.start(blockIdx.x), p1 = wk.start(blockIdx.x + 1);
@@ -199,14 +199,14 @@ cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int gri
   return cudaGetLastError();
 }
 
-int attend_hits_grid(int U, int k, int tail_split, int want) {
-  const long long V = (long long)U * (k + tail_split);
+int attend_hits_grid(int U, int vpu, int want) {
+  const long long V = (long long)U * vpu;
   if (want > V) want = (int)V;
   return want < 1 ? 1 : want;
 }
 
-int attend_hits_parts(int U, int k, int tail_split, int grid) {
-  return hits_segments_per_unit(U, k + tail_split, attend_hits_grid(U, k, tail_split, grid));
+int attend_hits_parts(int U, int vpu, int grid) {
+  return hits_segments_per_unit(U, vpu, attend_hits_grid(U, vpu, grid));
 }
 
 }  // namespace nosa

@@ -273,12 +273,17 @@ __device__ void contribute_partial(const DecodeArgs& a, int u, int n_seg, int n_
 }
 
 // The hits pass walks a virtual sequence of positions: unit u owns positions
-// [u * vpu, (u + 1) * vpu), vpu = k + tail_split; position j < k of unit u is
-// its j-th selected block (valid when j < k with KV resident, j < n_hit[u]
-// otherwise) and position k is its open tail (valid when it holds tokens).
+// [u * vpu, (u + 1) * vpu), vpu = k + tail_split + gap; position j < k of unit
+// u is its j-th selected block (valid when j < k with KV resident, j <
+// n_hit[u] otherwise), position k its open tail when tail_split is set (valid
+// when it holds tokens), and the gap positions after them are never valid.
 // CTA c takes the contiguous range [start(c), start(c + 1)), start(c) =
 // floor(c * V / grid), so every CTA streams the same number of positions and
 // touches one to a few units; each (unit, CTA) segment writes one partial.
+// Ending a segment in mid-range (storing the partial, counting it, loading
+// the next unit's queries) costs a CTA about as long as streaming a few
+// blocks; the gap charges that time to the CTAs whose range crosses a unit
+// boundary, which then stream fewer blocks.
 struct Walk {
   long long V;
   int vpu, grid;
@@ -294,7 +299,7 @@ struct Walk {
 // for it this step.
 __device__ __forceinline__ int hits_segments(const DecodeArgs& a, int u) {
   Walk wk;
-  wk.vpu = a.k + a.tail_split;
+  wk.vpu = a.vpu;
   wk.V = (long long)a.U * wk.vpu;
   wk.grid = a.hits_grid;
   return wk.segments(u);

@@ -148,8 +148,9 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
 
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = attend_hits_grid((int)U, k_sel, 0, 2 * sms);
-  const int nparts = attend_hits_parts((int)U, k_sel, 0, grid);
+  const int vpu = k_sel + kHitsGap;  // no open tail
+  const int grid = attend_hits_grid((int)U, vpu, 2 * sms);
+  const int nparts = attend_hits_parts((int)U, vpu, grid);
   if (U * nparts * G > kNoAllocRows)
     return noalloc_fail(NOSA_ERR_INVALID, "%lld partial rows exceed the fixed scratch of %d rows",
                         U * nparts * G, kNoAllocRows);
@@ -181,6 +182,7 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
   a.max_blocks = max_blocks;
   a.resident = 1;
   a.tail_split = 0;
+  a.vpu = vpu;
   a.part_base = 0;
   a.nparts = nparts;
   a.hits_grid = grid;

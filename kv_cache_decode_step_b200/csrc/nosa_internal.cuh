@@ -297,6 +297,7 @@ struct DecodeArgs {
   int U, Hq, Hkv, G, k, max_blocks, C;
   int resident;             // 1: sel indexes the resident KV
   int tail_split;           // 1: each unit's open tail is attended in the hits pass
+  int vpu;                  // hits-pass positions per unit: k + tail_split + the gap (kHitsGap)
   int part_base, nparts;    // hits pass writes slots part_base + segment; nparts per unit
   int miss_base;            // slot of a unit's first fetched-block partial
   int hits_grid;            // CTAs of the hits pass (fixes each unit's segment count)
@@ -314,9 +315,11 @@ struct DecodeMaps {
 cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st,
                                int stages = 3);
 // The hits-pass grid for a requested CTA count (at most one CTA per position).
-int attend_hits_grid(int U, int k, int tail_split, int want);
+int attend_hits_grid(int U, int vpu, int want);
 // Partial slots per unit the hits pass writes for this shape and requested grid.
-int attend_hits_parts(int U, int k, int tail_split, int want);
+int attend_hits_parts(int U, int vpu, int want);
+// Empty positions after each unit's blocks (and tail) in the hits pass walk.
+constexpr int kHitsGap = 3;
 // Kernel attributes (shared memory) of the attention kernels; once per device.
 cudaError_t configure_decode();
 cudaError_t configure_gather_attend();

@@ -156,6 +156,19 @@ def test_two_stage_hits_pass(offloaded, monkeypatch):
     _full(w, range(w.units), range(w.steps), cache_steps=[w.steps - 1] if offloaded else ())
 
 
+@pytest.mark.parametrize("gap", [0, 17])
+@pytest.mark.parametrize("offloaded", [True, False])
+def test_hits_pass_walk_gap(gap, offloaded, monkeypatch):
+    """The hits pass with no empty positions after each unit, and with more
+    empty positions than a unit has blocks (NOSA_ATTN_GAP): ranges that hold
+    only empty positions still count their segments."""
+    monkeypatch.setenv("NOSA_ATTN_GAP", str(gap))
+    w = configs.get("tiny", steps=8)
+    if not offloaded:
+        w = w.with_(offloaded=False, cache_factor=0)
+    _full(w, range(w.units), range(w.steps), cache_steps=[w.steps - 1] if offloaded else ())
+
+
 @pytest.mark.parametrize("graph", [False, True])
 def test_cache_of_exactly_k_slots(graph):
     """C = k: a full cache holds exactly S(t-1), so every miss evicts a block
