@@ -9,9 +9,12 @@
  *   nosa_score_blocks   block scores from pooled keys        (§3.1)
  *   nosa_select         eviction-bounded query-agnostic set + capped
  *                       query-aware top-k, overlap >= m       (§3.1, App. E)
- *   nosa_fetch_missing  set difference against the GPU block cache and a
- *                       zero-copy gather of the misses over PCIe (§4)
- *   nosa_sparse_decode  GQA attention over the selected blocks (App. A)
+ *   nosa_fetch_missing  set difference against the GPU block cache: which
+ *                       blocks miss and which slots they take (§4); it moves
+ *                       no bytes
+ *   nosa_sparse_decode  the zero-copy gather of the misses over PCIe (§4),
+ *                       fused with the GQA attention over the selected
+ *                       blocks (App. A)
  *
  * plus nosa_append_token first when the sequence grows during decoding.
  * nosa_score_select_fetch makes the first three calls in one (fused below
@@ -142,6 +145,11 @@ NOSA_API nosa_status nosa_attach_kv(nosa_ctx* ctx, const void* k, const void* v,
                            const float* agnostic, nosa_stream_t stream);
 
 /* Append one token per unit to the open tail block (first call of a step).
+ * NOSA summary App. A describes one decode step over a context that grows by
+ * the token just decoded; the reading here is that its K/V join an open tail
+ * block that is attended in full but neither scored nor fetched until its 64
+ * tokens close it, after which it is an ordinary candidate block (pooled keys
+ * as in §3.1, agnostic score as passed, stored on the host as in §1).
  * k_new, v_new: device bf16 [B, H_kv, d].  agnostic_if_close: device fp32 [U]
  * or NULL; it becomes the agnostic score of the tail block if this token fills
  * it, in which case nosa_sparse_decode closes the block at the end of the step
@@ -179,7 +187,9 @@ NOSA_API nosa_status nosa_score_blocks(nosa_ctx* ctx, const void* q, double* sco
  * nosa_score_blocks.  sel: device int32 [U, k], S(t) ascending, -1 padded. */
 NOSA_API nosa_status nosa_select(nosa_ctx* ctx, const double* scores, int32_t* sel, nosa_stream_t stream);
 
-/* Cache planning and miss gather (NOSA summary §4, App. A).  Per unit the
+/* Cache planning (NOSA summary §4, App. A).  This call plans only: it moves
+ * no bytes, and when its stream has drained the missed blocks are still in
+ * host memory; nosa_sparse_decode copies them.  Per unit the
  * misses M = S(t) \ R(t-1) (R = blocks resident in the GPU cache) get slots:
  * free slots first (lowest first), then resident blocks outside S(t), least
  * recently selected first, lower block id on ties.  Only blocks unused by this
@@ -230,19 +240,31 @@ NOSA_API nosa_status nosa_sparse_decode(nosa_ctx* ctx, const void* q, const int3
  * for each query head h of unit u, out_h = softmax(q_h K^T / sqrt(d)) V over the
  * 64 tokens of each block listed in sel[u].  q: device bf16 [B, H_q, 128];
  * k, v: device bf16 [U, max_blocks*64, 128], 16-byte aligned; sel: device
- * int32 [U, k_sel] of valid block ids (an out-of-range id reads block 0);
- * out: device bf16 [B, H_q, 128].  Split-KV partials live in a fixed array
- * inside the library (8.5 MB per GPU that loads it, held until exit): the call
- * returns NOSA_ERR_INVALID when B*H_q exceeds 8192 query heads.
+ * int32 [U, k_sel] of block ids (an out-of-range id is flagged and block 0 is
+ * read in its place); out: device bf16 [B, H_q, 128].  With the same inputs the
+ * output is bit-identical to nosa_sparse_decode's over resident KV.  Split-KV
+ * partials live in a fixed array inside the library (8.5 MB per GPU that loads
+ * it, held until exit): the call returns NOSA_ERR_INVALID when B*H_q exceeds
+ * 8192 query heads.
  * The first call on a device resolves that array's device address (once per
  * device, with the device current), so make it before any stream capture.
  * Every call shares the array and leaves its contents behind; each call
- * clears the small status word it needs and fully writes the partials it
- * reads, but calls that overlap on the GPU (on different streams) race. */
+ * clears the merge counters it needs and fully writes the partials it reads,
+ * but calls that overlap on the GPU (on different streams) race.  Device-side
+ * errors (an out-of-range id, a bounded wait that ran out and left outputs
+ * unwritten) are not returned by this asynchronous call: they accumulate in a
+ * per-device error word that nosa_noalloc_check_errors reports. */
 NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, const void* v, int batch,
                                                 int n_q_heads, int n_kv_heads, int max_blocks,
                                                 const int32_t* sel, int k_sel, void* out,
                                                 nosa_stream_t stream);
+
+/* Synchronous (waits for stream).  Reports and clears the error word that
+ * nosa_sparse_decode_noalloc calls on the current device have set since the
+ * last check: NOSA_ERR_TIMEOUT when a bounded device wait ran out (that call's
+ * outputs are incomplete), NOSA_ERR_INVALID when a selected block id was out of
+ * range, else NOSA_OK.  Allocates nothing. */
+NOSA_API nosa_status nosa_noalloc_check_errors(nosa_stream_t stream);
 
 /* Row gather at a chosen granularity (NOSA summary §3.2 and §4: block-wise
  * transfer of 16 KiB blocks against element-wise transfer of single tokens).
@@ -264,6 +286,19 @@ NOSA_API nosa_status nosa_gather_rows(const void* src, int64_t src_rows, void* d
                                       int32_t row_bytes, const int64_t* src_idx, const int64_t* dst_idx,
                                       int32_t n, int32_t ctas, uint32_t* flags, nosa_stream_t stream);
 
+/* The row gather of nosa_gather_rows (same arguments, result and errors)
+ * through the TMA unit instead of SM loads: every row, or 16 KiB piece of a
+ * longer row, is one asynchronous bulk copy into shared memory (completing
+ * on an mbarrier) and one bulk copy out to dst.  It is the transfer study's
+ * second arm (NOSA summary §4: a dedicated transfer kernel over 16 KiB blocks
+ * through unified virtual addressing): the bulk copies issue their own PCIe
+ * read requests.  ctas: CTAs of 4 copying warps, 0 for a quarter of the SMs.
+ * flags bit 1 is ORed in when a copy did not complete within about 1 s (the
+ * kernel stops early; the context of the caller stays usable). */
+NOSA_API nosa_status nosa_gather_rows_bulk(const void* src, int64_t src_rows, void* dst, int64_t dst_rows,
+                                           int32_t row_bytes, const int64_t* src_idx, const int64_t* dst_idx,
+                                           int32_t n, int32_t ctas, uint32_t* flags, nosa_stream_t stream);
+
 /* Synchronous.  Copies the running totals into *stats. */
 NOSA_API nosa_status nosa_get_stats(nosa_ctx* ctx, nosa_stats* stats);
 
@@ -280,6 +315,15 @@ NOSA_API nosa_status nosa_check_errors(nosa_ctx* ctx);
  * slot, -1 if free.  NOSA_ERR_INVALID when KV is resident. */
 NOSA_API nosa_status nosa_read_cache_map(nosa_ctx* ctx, int32_t* slot_block);
 
+/* Synchronous.  Copies the GPU block cache of units [unit_begin,
+ * unit_begin + n_units) into host buffers k_host, v_host, each bf16
+ * [n_units, cache_slots, P, d]: slot s of a unit holds the K (V) rows of the
+ * block nosa_read_cache_map names for it (contents of free slots are
+ * unspecified).  For checking the miss gather (NOSA summary §4: the missed
+ * blocks land in their GPU slots).  NOSA_ERR_INVALID when KV is resident or
+ * the range is outside [0, U). */
+NOSA_API nosa_status nosa_read_cache(nosa_ctx* ctx, int unit_begin, int n_units, void* k_host, void* v_host);
+
 /* Synchronous checkpoint of the decode state: step counter, block count,
  * Gamma_e, S(t-1), cache tables, agnostic scores and the open tail block.
  * Pass buf = NULL to query the size in *size.  Cache contents and pooled keys
@@ -295,6 +339,15 @@ NOSA_API nosa_status nosa_set_state(nosa_ctx* ctx, const void* buf, size_t size)
  * and returns, leaving the context usable. */
 NOSA_API nosa_status nosa_debug_wait_flag(nosa_ctx* ctx, const int32_t* flag, int timeout_ms,
                                  nosa_stream_t stream);
+
+/* Diagnostic: inject one host-side CUDA failure on the calling thread.  The
+ * context calls (nosa_create ... nosa_set_state) check every CUDA runtime call
+ * they make; after this call the check that follows `skip` further checks is
+ * not made at all and reports cudaErrorLaunchFailure instead, so that call
+ * returns NOSA_ERR_CUDA.  Nothing reaches the GPU.  The work the failed call
+ * enqueued before the failure still runs; nosa_attach_kv brings the context
+ * back to a clean step 0.  skip = -1 cancels a pending injection. */
+NOSA_API nosa_status nosa_debug_inject_cuda_error(int skip);
 
 /* Message of the last failure on the calling thread ("" if none). */
 NOSA_API const char* nosa_last_error(void);

@@ -34,9 +34,20 @@ nosa_status fail(nosa_status s, const char* fmt, ...) {
   return s;
 }
 
+// Injected host-side failures (nosa_debug_inject_cuda_error): the checked
+// CUDA call that follows `g_inject_skip` further checked calls on this thread
+// is not made and reports cudaErrorLaunchFailure.  -1: off.
+thread_local int g_inject_skip = -1;
+
+bool inject_now() {
+  if (g_inject_skip < 0) return false;
+  if (g_inject_skip-- > 0) return false;
+  return true;  // g_inject_skip is now -1: one failure only
+}
+
 #define NOSA_CUDA(call)                                                                   \
   do {                                                                                    \
-    cudaError_t e_ = (call);                                                              \
+    cudaError_t e_ = inject_now() ? cudaErrorLaunchFailure : (call);                      \
     if (e_ != cudaSuccess) {                                                              \
       return fail(e_ == cudaErrorMemoryAllocation ? NOSA_ERR_NOMEM : NOSA_ERR_CUDA,       \
                   "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__,      \
@@ -802,6 +813,21 @@ nosa_status nosa_read_cache_map(nosa_ctx* c, int32_t* slot_block) {
   return NOSA_OK;
 }
 
+nosa_status nosa_read_cache(nosa_ctx* c, int unit_begin, int n_units, void* k_host, void* v_host) {
+  if (!c || !k_host || !v_host) return fail(NOSA_ERR_INVALID, "ctx, k_host and v_host must be non-NULL");
+  if (!c->offloaded) return fail(NOSA_ERR_INVALID, "KV is resident: there is no cache");
+  if (unit_begin < 0 || n_units < 0 || unit_begin + (long long)n_units > c->U)
+    return fail(NOSA_ERR_INVALID, "units [%d, %d + %d) outside [0, %d)", unit_begin, unit_begin, n_units, c->U);
+  nosa_status s = set_device(c);
+  if (s != NOSA_OK) return s;
+  NOSA_CUDA(cudaDeviceSynchronize());
+  const size_t per_unit = (size_t)c->C * kP * kD;  // bf16 elements of one unit's slots
+  const size_t bytes = per_unit * n_units * sizeof(uint16_t);
+  NOSA_CUDA(cudaMemcpy(k_host, c->cache_k + per_unit * unit_begin, bytes, cudaMemcpyDeviceToHost));
+  NOSA_CUDA(cudaMemcpy(v_host, c->cache_v + per_unit * unit_begin, bytes, cudaMemcpyDeviceToHost));
+  return NOSA_OK;
+}
+
 // ---------------------------------------------------------------- checkpoint
 namespace {
 struct StateHeader {
@@ -949,6 +975,12 @@ nosa_status nosa_set_state(nosa_ctx* c, const void* buf, size_t size) {
   c->h_appended = false;
   c->appends_enabled = c->appends_enabled || d.tail_len > 0;
   c->phase = kReady;
+  return NOSA_OK;
+}
+
+nosa_status nosa_debug_inject_cuda_error(int skip) {
+  if (skip < -1) return fail(NOSA_ERR_INVALID, "skip must be >= -1");
+  g_inject_skip = skip;
   return NOSA_OK;
 }
 

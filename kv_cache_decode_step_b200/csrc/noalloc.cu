@@ -148,7 +148,11 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
 
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int vpu = k_sel + kHitsGap;  // no open tail
+  // The walk of a context over resident KV: k blocks, a tail position (never
+  // valid here: there is no open tail) and the gap.  With the same grid the
+  // CTAs cover the same blocks and write the same partials, so the output is
+  // bit-identical to nosa_sparse_decode's on the same inputs.
+  const int vpu = k_sel + 1 + kHitsGap;
   const int grid = attend_hits_grid((int)U, vpu, 2 * sms);
   const int nparts = attend_hits_parts((int)U, vpu, grid);
   if (U * nparts * G > kNoAllocRows)
@@ -162,9 +166,9 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
   maps.tv = maps.v;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  e = cudaMemsetAsync(ds->state, 0, sizeof(DevState), st);
-  if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
-
+  // the merge counters must start at zero (a call stopped by a timeout leaves
+  // them behind); the error word is left alone: it accumulates until
+  // nosa_noalloc_check_errors reads and clears it
   e = cudaMemsetAsync(ds->unit_done, 0, (size_t)U * sizeof(int), st);
   if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
 
@@ -190,6 +194,28 @@ NOSA_API nosa_status nosa_sparse_decode_noalloc(const void* q, const void* k, co
   a.out = static_cast<uint16_t*>(out);
   e = launch_attend_hits(a, maps, grid, st);
   if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
+  return NOSA_OK;
+}
+
+NOSA_API nosa_status nosa_noalloc_check_errors(nosa_stream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  DeviceScratch* ds = nullptr;
+  nosa_status s = device_scratch(dev, &ds);
+  if (s != NOSA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned bits = 0;
+  e = cudaMemcpyAsync(&bits, &ds->state->error_bits, sizeof bits, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(&ds->state->error_bits, 0, sizeof bits, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return noalloc_fail(NOSA_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+  if (bits & ERR_TIMEOUT)
+    return noalloc_fail(NOSA_ERR_TIMEOUT, "a bounded device wait ran out (bits 0x%x): outputs of that call are "
+                        "incomplete", bits);
+  if (bits)
+    return noalloc_fail(NOSA_ERR_INVALID, "a selected block id was out of range (bits 0x%x): block 0 was read "
+                        "in its place", bits);
   return NOSA_OK;
 }
 

@@ -72,6 +72,92 @@ __global__ void __launch_bounds__(kRowsThreads) gather_rows_kernel(RowsArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- bulk copies
+// The same row gather through the TMA unit: each row (or 16 KiB piece of a
+// longer row) is one cp.async.bulk global -> shared load, completing on an
+// mbarrier, then one cp.async.bulk shared -> global store.  Every warp is an
+// independent copier whose lane 0 keeps up to kBulkSlots pieces in flight in
+// its own ring of shared-memory slots.  The copy engine of the TMA unit issues
+// its own memory requests, so the PCIe read requests are not shaped by 16-byte
+// SM loads.
+constexpr int kBulkThreads = 128;
+constexpr int kBulkWarps = kBulkThreads / 32;
+constexpr int kBulkSlots = 8;                  // most pieces in flight per warp
+constexpr int kBulkRingBytes = 48 * 1024;      // shared memory per warp
+constexpr int kBulkSmemBytes = 1024 + kBulkWarps * kBulkRingBytes;
+constexpr int kBulkPieceMax = 16384;
+constexpr uint64_t kBulkWaitNs = 1000000000ull;
+
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(gdst)),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// a.total counts pieces here, log_piece = log2(piece bytes), a.log_cpr =
+// log2(pieces per row); nslots = min(kBulkSlots, kBulkRingBytes / piece).
+__global__ void __launch_bounds__(kBulkThreads) gather_rows_bulk_kernel(RowsArgs a, int log_piece, int nslots) {
+  extern __shared__ __align__(1024) unsigned char bulk_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane != 0) return;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bulk_smem) + warp * kBulkSlots;
+  unsigned char* ring = bulk_smem + 1024 + warp * kBulkRingBytes;
+  const uint32_t piece = 1u << log_piece;
+  for (int s = 0; s < nslots; ++s) mbar_init(&bars[s], 1);
+  fence_mbar_init();
+  const long long agents = (long long)gridDim.x * kBulkWarps;
+  const long long mask = (1ll << a.log_cpr) - 1;
+  const unsigned char* src = reinterpret_cast<const unsigned char*>(a.src);
+  unsigned char* dst = reinterpret_cast<unsigned char*>(a.dst);
+  long long next = (long long)blockIdx.x * kBulkWarps + warp;  // next piece this warp considers
+  long long dst_off[kBulkSlots];
+  int head = 0, tail = 0;  // pieces loaded (issued), pieces stored
+  // issue the next in-range piece into slot head % nslots; false when none is left
+  auto issue = [&]() -> bool {
+    while (next < a.total) {
+      const long long c = next;
+      next += agents;
+      const long long row = c >> a.log_cpr;
+      const long long s = __ldg(a.src_idx + row);
+      const long long t = a.dst_idx ? __ldg(a.dst_idx + row) : row;
+      if (s < 0 || s >= a.src_rows || t < 0 || t >= a.dst_rows) {
+        if (a.flags) atomicOr(a.flags, 1u);
+        continue;
+      }
+      const int slot = head % nslots;
+      const long long off = (c & mask) << log_piece;
+      dst_off[slot] = ((t << a.log_cpr) << log_piece) + off;
+      mbar_arrive_expect_tx(&bars[slot], piece);
+      bulk_load(ring + (size_t)slot * piece, src + ((s << a.log_cpr) << log_piece) + off, piece, &bars[slot]);
+      ++head;
+      return true;
+    }
+    return false;
+  };
+  while (head < nslots && issue()) {
+  }
+  while (tail < head) {
+    const int slot = tail % nslots;
+    if (!mbar_wait_bounded(&bars[slot], (uint32_t)((tail / nslots) & 1), kBulkWaitNs)) {
+      // record, give the other loads in flight a bounded chance to land, stop
+      if (a.flags) atomicOr(a.flags, 2u);
+      for (int g = tail + 1; g < head; ++g)
+        (void)mbar_wait_bounded(&bars[g % nslots], (uint32_t)((g / nslots) & 1), kBulkWaitNs);
+      break;
+    }
+    bulk_store(dst + dst_off[slot], ring + (size_t)slot * piece, piece);
+    ++tail;
+    // the slot of the piece just stored is reloaded once the store has read it
+    bulk_wait_read_all();
+    issue();
+  }
+  bulk_wait_all();
+}
+
 nosa_status rows_fail(nosa_status s, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -85,18 +171,20 @@ nosa_status rows_fail(nosa_status s, const char* fmt, ...) {
 }  // namespace
 }  // namespace nosa
 
-using namespace nosa;
+namespace nosa {
+namespace {
 
-extern "C" {
-
-NOSA_API nosa_status nosa_gather_rows(const void* src, int64_t src_rows, void* dst, int64_t dst_rows,
-                                      int32_t row_bytes, const int64_t* src_idx, const int64_t* dst_idx,
-                                      int32_t n, int32_t ctas, uint32_t* flags, nosa_stream_t stream) {
+// Validation and argument set-up shared by both gathers; *grid is the CTA
+// count asked for (0: a quarter of the SMs).
+nosa_status rows_setup(const void* src, int64_t src_rows, void* dst, int64_t dst_rows, int32_t row_bytes,
+                       const int64_t* src_idx, const int64_t* dst_idx, int32_t n, int32_t ctas, uint32_t* flags,
+                       RowsArgs* a, int* grid) {
   if (n < 0) return rows_fail(NOSA_ERR_INVALID, "n = %d < 0", n);
   if (row_bytes < 16 || row_bytes > 65536 || (row_bytes & (row_bytes - 1)) != 0)
     return rows_fail(NOSA_ERR_INVALID, "row_bytes = %d is not a power of two in [16, 65536]", row_bytes);
   if (ctas < 0 || ctas > 65535) return rows_fail(NOSA_ERR_INVALID, "ctas = %d outside [0, 65535]", ctas);
   if (src_rows < 0 || dst_rows < 0) return rows_fail(NOSA_ERR_INVALID, "negative row counts");
+  *grid = 0;
   if (n == 0) return NOSA_OK;
   if (!src || !dst || !src_idx) return rows_fail(NOSA_ERR_INVALID, "NULL argument");
   if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % 16 != 0)
@@ -116,32 +204,79 @@ NOSA_API nosa_status nosa_gather_rows(const void* src, int64_t src_rows, void* d
   while ((16 << log_cpr) < row_bytes) ++log_cpr;
   if (src_rows > (1ll << 59 >> log_cpr) || dst_rows > (1ll << 59 >> log_cpr))
     return rows_fail(NOSA_ERR_INVALID, "row counts too large");
-
-  int grid = ctas;
-  if (grid == 0) {
+  int g = ctas;
+  if (g == 0) {
     int dev = 0, sms = 148;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return rows_fail(NOSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    grid = (sms + 3) / 4;
+    g = (sms + 3) / 4;
   }
-  const long long total = (long long)n << log_cpr;
-  const long long need = (total + kRowsThreads * kRowsUnroll - 1) / (kRowsThreads * kRowsUnroll);
-  if (grid > need) grid = (int)need;
+  *a = RowsArgs{};
+  a->src = static_cast<const uint4*>(src_dev);
+  a->dst = static_cast<uint4*>(dst_dev);
+  a->src_idx = src_idx;
+  a->dst_idx = dst_idx;
+  a->src_rows = src_rows;
+  a->dst_rows = dst_rows;
+  a->total = (long long)n << log_cpr;
+  a->log_cpr = log_cpr;
+  a->flags = flags;
+  *grid = g;
+  return NOSA_OK;
+}
 
-  RowsArgs a{};
-  a.src = static_cast<const uint4*>(src_dev);
-  a.dst = static_cast<uint4*>(dst_dev);
-  a.src_idx = src_idx;
-  a.dst_idx = dst_idx;
-  a.src_rows = src_rows;
-  a.dst_rows = dst_rows;
-  a.total = total;
-  a.log_cpr = log_cpr;
-  a.flags = flags;
+}  // namespace
+}  // namespace nosa
+
+using namespace nosa;
+
+extern "C" {
+
+NOSA_API nosa_status nosa_gather_rows(const void* src, int64_t src_rows, void* dst, int64_t dst_rows,
+                                      int32_t row_bytes, const int64_t* src_idx, const int64_t* dst_idx,
+                                      int32_t n, int32_t ctas, uint32_t* flags, nosa_stream_t stream) {
+  RowsArgs a;
+  int grid = 0;
+  nosa_status s = rows_setup(src, src_rows, dst, dst_rows, row_bytes, src_idx, dst_idx, n, ctas, flags, &a, &grid);
+  if (s != NOSA_OK || grid == 0) return s;
+  const long long need = (a.total + kRowsThreads * kRowsUnroll - 1) / (kRowsThreads * kRowsUnroll);
+  if (grid > need) grid = (int)need;
   gather_rows_kernel<<<grid, kRowsThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return rows_fail(NOSA_ERR_CUDA, "gather launch: %s", cudaGetErrorString(e));
+  return NOSA_OK;
+}
+
+NOSA_API nosa_status nosa_gather_rows_bulk(const void* src, int64_t src_rows, void* dst, int64_t dst_rows,
+                                           int32_t row_bytes, const int64_t* src_idx, const int64_t* dst_idx,
+                                           int32_t n, int32_t ctas, uint32_t* flags, nosa_stream_t stream) {
+  RowsArgs a;
+  int grid = 0;
+  nosa_status s = rows_setup(src, src_rows, dst, dst_rows, row_bytes, src_idx, dst_idx, n, ctas, flags, &a, &grid);
+  if (s != NOSA_OK || grid == 0) return s;
+  // pieces of at most 16 KiB: a.total and a.log_cpr count pieces, not 16-byte words
+  int log_piece = 4;
+  while ((1 << log_piece) < row_bytes && (2 << log_piece) <= kBulkPieceMax) ++log_piece;
+  int log_rb = 4;
+  while ((1 << log_rb) < row_bytes) ++log_rb;
+  a.log_cpr = log_rb - log_piece;
+  a.total = (long long)n << a.log_cpr;
+  int nslots = kBulkRingBytes >> log_piece;
+  if (nslots > kBulkSlots) nslots = kBulkSlots;
+  const long long need = (a.total + kBulkWarps - 1) / kBulkWarps;
+  if (grid > need) grid = (int)need;
+  static bool configured = false;  // per process; the attribute is per device function
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gather_rows_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kBulkSmemBytes);
+    if (e != cudaSuccess) return rows_fail(NOSA_ERR_CUDA, "bulk gather configuration: %s", cudaGetErrorString(e));
+    configured = true;
+  }
+  gather_rows_bulk_kernel<<<grid, kBulkThreads, kBulkSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(
+      a, log_piece, nslots);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return rows_fail(NOSA_ERR_CUDA, "bulk gather launch: %s", cudaGetErrorString(e));
   return NOSA_OK;
 }
 

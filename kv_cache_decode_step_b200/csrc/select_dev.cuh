@@ -12,12 +12,15 @@ namespace nosa {
 constexpr unsigned kFull = 0xffffffffu;
 
 // Order-preserving maps to unsigned integers.  No real key maps to 0, which
-// marks "no candidate".
+// marks "no candidate".  -0.0 and +0.0 compare equal, so both map to the key
+// of +0.0 and their order falls to the block ids like any other tie.
 __device__ __forceinline__ unsigned long long key_f64(double x) {
+  if (x == 0.0) x = 0.0;
   const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
   return (b & 0x8000000000000000ull) ? ~b : (b | 0x8000000000000000ull);
 }
 __device__ __forceinline__ unsigned long long key_f32(float x) {
+  if (x == 0.0f) x = 0.0f;
   const unsigned b = __float_as_uint(x);
   return (unsigned long long)((b & 0x80000000u) ? ~b : (b | 0x80000000u)) << 32;
 }

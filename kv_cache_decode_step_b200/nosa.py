@@ -31,7 +31,8 @@ ENTRY_POINTS = (
     "nosa_select", "nosa_fetch_missing", "nosa_sparse_decode", "nosa_get_stats", "nosa_reset_stats",
     "nosa_check_errors", "nosa_read_cache_map", "nosa_get_state", "nosa_set_state",
     "nosa_debug_wait_flag", "nosa_last_error", "nosa_version", "nosa_sparse_decode_noalloc",
-    "nosa_gather_rows", "nosa_score_select_fetch",
+    "nosa_gather_rows", "nosa_score_select_fetch", "nosa_gather_rows_bulk", "nosa_noalloc_check_errors",
+    "nosa_read_cache", "nosa_debug_inject_cuda_error",
 )
 
 
@@ -92,7 +93,11 @@ def lib() -> C.CDLL:
             "nosa_last_error": ([], C.c_char_p),
             "nosa_version": ([], C.c_char_p),
             "nosa_sparse_decode_noalloc": ([vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp], st),
+            "nosa_noalloc_check_errors": ([vp], st),
+            "nosa_read_cache": ([vp, i32, i32, vp, vp], st),
+            "nosa_debug_inject_cuda_error": ([i32], st),
             "nosa_gather_rows": ([vp, C.c_int64, vp, C.c_int64, i32, vp, vp, i32, i32, vp, vp], st),
+            "nosa_gather_rows_bulk": ([vp, C.c_int64, vp, C.c_int64, i32, vp, vp, i32, i32, vp, vp], st),
             "nosa_score_select_fetch": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
         }
         for name, (args, res) in sig.items():
@@ -203,6 +208,14 @@ def nosa_read_cache_map(ctx, out) -> None:
     _check(lib().nosa_read_cache_map(ctx, _ptr(out)), "nosa_read_cache_map")
 
 
+def nosa_read_cache(ctx, unit_begin: int, n_units: int, k_out, v_out) -> None:
+    _check(lib().nosa_read_cache(ctx, int(unit_begin), int(n_units), _ptr(k_out), _ptr(v_out)), "nosa_read_cache")
+
+
+def nosa_debug_inject_cuda_error(skip: int) -> None:
+    _check(lib().nosa_debug_inject_cuda_error(int(skip)), "nosa_debug_inject_cuda_error")
+
+
 def nosa_get_state(ctx) -> bytes:
     size = C.c_size_t(0)
     _check(lib().nosa_get_state(ctx, None, C.byref(size)), "nosa_get_state")
@@ -228,11 +241,22 @@ def nosa_sparse_decode_noalloc(q, k, v, batch: int, n_q_heads: int, n_kv_heads: 
                                             _ptr(out), _stream(stream)), "nosa_sparse_decode_noalloc")
 
 
+def nosa_noalloc_check_errors(stream=None) -> None:
+    _check(lib().nosa_noalloc_check_errors(_stream(stream)), "nosa_noalloc_check_errors")
+
+
 def nosa_gather_rows(src, src_rows: int, dst, dst_rows: int, row_bytes: int, src_idx, dst_idx, n: int,
                      ctas: int = 0, flags=None, stream=None) -> None:
     _check(lib().nosa_gather_rows(_ptr(src), int(src_rows), _ptr(dst), int(dst_rows), int(row_bytes),
                                   _ptr(src_idx), _ptr(dst_idx), int(n), int(ctas), _ptr(flags),
                                   _stream(stream)), "nosa_gather_rows")
+
+
+def nosa_gather_rows_bulk(src, src_rows: int, dst, dst_rows: int, row_bytes: int, src_idx, dst_idx, n: int,
+                          ctas: int = 0, flags=None, stream=None) -> None:
+    _check(lib().nosa_gather_rows_bulk(_ptr(src), int(src_rows), _ptr(dst), int(dst_rows), int(row_bytes),
+                                       _ptr(src_idx), _ptr(dst_idx), int(n), int(ctas), _ptr(flags),
+                                       _stream(stream)), "nosa_gather_rows_bulk")
 
 
 def config_from_workload(w) -> nosa_config:

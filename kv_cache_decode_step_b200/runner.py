@@ -108,8 +108,10 @@ class Decoder:
 
     # ------------------------------------------------------------ one step
     def _load_inputs(self, t: int) -> None:
-        """Copy step t's inputs into the static buffers (on self.stream)."""
-        self.q.copy_(self.q_all[t], non_blocking=True)
+        """Copy step t's inputs into the static buffers (on self.stream).
+        Queries are reused cyclically past the workload's last step (a run
+        longer than the workload); appended tokens are not."""
+        self.q.copy_(self.q_all[t % self.q_all.shape[0]], non_blocking=True)
         if self.w.append:
             self.k_in.copy_(self.k_new[t], non_blocking=True)
             self.v_in.copy_(self.v_new[t], non_blocking=True)
@@ -159,6 +161,17 @@ class Decoder:
         out = np.zeros((self.w.units, self.w.cache_slots), dtype=np.int32)
         nosa.nosa_read_cache_map(self.ctx, out)
         return out
+
+    def cache_contents(self, unit_begin: int = 0, n_units: Optional[int] = None):
+        """K and V of every cache slot of the given units: uint16 (bf16 bits)
+        [n_units, cache_slots, block, head_dim] each."""
+        w = self.w
+        n_units = w.units - unit_begin if n_units is None else n_units
+        shape = (n_units, w.cache_slots, w.block, w.head_dim)
+        k = np.zeros(shape, dtype=np.uint16)
+        v = np.zeros(shape, dtype=np.uint16)
+        nosa.nosa_read_cache(self.ctx, unit_begin, n_units, k, v)
+        return k, v
 
     def check(self) -> None:
         nosa.nosa_check_errors(self.ctx)

@@ -6,7 +6,7 @@ batch 64, sequence length 4096, d_kv = 128 and 2 KV heads, as locality rises;
 §4 describes the block transfer as a zero-copy kernel over 16 KiB blocks.
 
 This module measures both with one kernel (``nosa_gather_rows``) on the same
-miss volume.  Per unit (sequence, KV head) the selection budget is 16 blocks
+miss volume, and again with TMA bulk copies (``nosa_gather_rows_bulk``).  Per unit (sequence, KV head) the selection budget is 16 blocks
 (1024 tokens, a quarter of the sequence); at locality gamma the step misses
 (1 - gamma) * 1024 tokens, i.e. 8, 4, 2 or 1 blocks for gamma = 0.5, 0.75,
 0.875, 0.9375.  Block-wise, each missed block is a 16 KiB row of K and one of
@@ -60,7 +60,8 @@ def miss_sets(rng, gamma: float, row_bytes: int, reps: int):
     return m, out
 
 
-def time_gathers(torch, host, cache, sets, row_bytes: int, ctas: int, flush, stream):
+def time_gathers(torch, host, cache, sets, row_bytes: int, ctas: int, flush, stream, fn=None):
+    fn = fn or nosa.nosa_gather_rows
     src_rows = host.numel() // row_bytes
     dst_rows = cache.numel() // row_bytes
     dev_sets = [(torch.from_numpy(s).cuda(), torch.from_numpy(d).cuda()) for s, d in sets]
@@ -72,8 +73,7 @@ def time_gathers(torch, host, cache, sets, row_bytes: int, ctas: int, flush, str
             flush.fill_(i & 0xFF)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            nosa.nosa_gather_rows(host, src_rows, cache, dst_rows, row_bytes, s, d, s.numel(), ctas, flags,
-                                  stream)
+            fn(host, src_rows, cache, dst_rows, row_bytes, s, d, s.numel(), ctas, flags, stream)
             e1.record(stream)
             if i >= 3:
                 ms.append((e0, e1))
@@ -154,6 +154,16 @@ def main(argv=None) -> int:
             m, sets = miss_sets(rng, gamma, rb, args.reps)
             record("gather_rows", gamma, rb, default_ctas, m,
                    time_gathers(torch, host, cache, sets, rb, default_ctas, flush, stream))
+            record("gather_rows_bulk", gamma, rb, default_ctas, m,
+                   time_gathers(torch, host, cache, sets, rb, default_ctas, flush, stream,
+                                nosa.nosa_gather_rows_bulk))
+    # the TMA bulk arm at other grid widths (block rows and token rows)
+    for g in (1, 64):
+        rb = g * TOKEN_BYTES
+        m, sets = miss_sets(rng, 0.75, rb, args.reps)
+        for ctas in (default_ctas // 2, 2 * default_ctas, sms, 2 * sms):
+            record("gather_rows_bulk", 0.75, rb, ctas, m,
+                   time_gathers(torch, host, cache, sets, rb, ctas, flush, stream, nosa.nosa_gather_rows_bulk))
     # rows below one token: where does the request size start to cost?
     for rb in SUB_TOKEN_ROWS:
         m, sets = miss_sets(rng, 0.75, rb, args.reps)

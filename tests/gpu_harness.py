@@ -56,12 +56,42 @@ def run_gpu(w, data, sample: Sequence[int], attend_steps, steps=None, graph=Fals
             if t in cache_steps and w.offloaded:
                 cm = dec.cache_map()
                 rec.resident[t] = [np.sort(cm[u][cm[u] >= 0]) for u in sample]
+                check_cache_bytes(w, data, dec, cm, sample, t)
         rec.sel_all_last = dec.sel.cpu().numpy()
         rec.stats = dec.stats()
         dec.check()
     finally:
         dec.close()
     return rec
+
+
+def check_cache_bytes(w, data, dec, cache_map, sample, t, chunk=64):
+    """Every occupied cache slot of the sampled units holds, byte for byte, the
+    K and V rows of the block the cache map names (the input arrays: prompt
+    rows, and for growing sequences the appended rows, which are the later rows
+    of the same per-unit streams)."""
+    P = w.block
+    sample = sorted(sample)
+    i = 0
+    while i < len(sample):
+        # contiguous runs of units, read in chunks
+        j = i
+        while j + 1 < len(sample) and sample[j + 1] == sample[j] + 1 and j + 1 - i < chunk:
+            j += 1
+        u0, n = sample[i], j - i + 1
+        ck, cv = dec.cache_contents(u0, n)
+        for du in range(n):
+            u = u0 + du
+            for slot, b in enumerate(cache_map[u]):
+                if b < 0:
+                    continue
+                for name, got, src in (("K", ck[du, slot], data["k"][u]), ("V", cv[du, slot], data["v"][u])):
+                    if not np.array_equal(got, src[b * P:(b + 1) * P]):
+                        bad = np.argwhere(got != src[b * P:(b + 1) * P])
+                        raise AssertionError(f"step {t} unit {u} slot {slot} block {b}: cached {name} differs "
+                                             f"from the host block at {len(bad)} of {got.size} elements, first "
+                                             f"(token, dim) {tuple(bad[0])}")
+        i = j + 1
 
 
 def run_oracle(w, data, sample, attend_steps, steps=None) -> List[oracle.UnitRun]:

@@ -1,8 +1,11 @@
 """GPU parity: the CUDA path, called through the C ABI, against the CPU oracle
 on the same seeded inputs.  Selections, fetch lists and resident sets must be
-bit-exact; bf16 attention outputs within max-abs 2e-2 and mean-abs 2e-3 of the
-oracle's fp64 result.  The five workloads run at full size (the oracle checks
-a sample of units, every step of their selections)."""
+bit-exact, and so must the bytes of every occupied cache slot (against the
+host block it names); bf16 attention outputs within max-abs 2e-2 and mean-abs
+2e-3 of the oracle's fp64 result.  The five workloads run at full size; on the
+offloaded batch-64 workload and the long-input workload every unit's
+selections and fetch lists are compared at every step, elsewhere a sample of
+units."""
 
 import numpy as np
 import pytest
@@ -37,15 +40,19 @@ def test_layer8b_resident():
 
 
 def test_offload_b64_graph_replay():
+    """Every unit: S(t), fetch lists and n_fetch at all 256 steps; resident
+    sets and cache bytes at three steps; outputs at nine."""
     w = configs.get("offload_b64")
-    _full(w, [0, 101, 256, 511], list(range(0, w.steps, 32)) + [w.steps - 1], graph=True,
+    _full(w, range(w.units), list(range(0, w.steps, 32)) + [w.steps - 1], graph=True,
           cache_steps=[1, 100, w.steps - 1])
 
 
 def test_long_input_offloaded():
+    """Every unit, every step; the query resamples (t % 32 == 0) push the
+    capped selection to its limit."""
     w = configs.get("long_input")
-    _full(w, [0, 13, 31], list(range(0, w.steps, 16)) + [31, 32, 33, w.steps - 1],
-          cache_steps=[31, 32, w.steps - 1])
+    _full(w, range(w.units), list(range(0, w.steps, 16)) + [31, 32, 33, w.steps - 1],
+          cache_steps=[0, 31, 32, 33, w.steps - 1])
 
 
 def test_long_generation_appends_and_closes():

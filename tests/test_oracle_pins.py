@@ -240,6 +240,17 @@ def test_ties_go_to_lowest_block_id(orc):
     assert orc.select(np.zeros(10), [9], [], True, 3, 0).tolist() == [0, 1, 2, 9]
 
 
+def test_signed_zeros_are_equal_scores(orc):
+    """-0.0 and +0.0 are the same value: their order falls to the block ids."""
+    a = np.array([0.0, -0.0, 0.0, -0.0, 1.0, -0.0], dtype=np.float32)
+    assert orc.evict_update(a, [], 0, 6, 3).tolist() == [0, 1, 4]
+    a2 = np.array([-0.0, 0.0, -0.0, 0.0, 1.0, 0.0], dtype=np.float32)
+    assert orc.evict_update(a2, [], 0, 6, 3).tolist() == [0, 1, 4]
+    s = np.array([-0.0, 0.0, -0.0, 2.0, 0.0])
+    assert orc.select(s, [], [], True, 2, 0).tolist() == [0, 3]
+    assert orc.select(-s, [], [], True, 2, 0).tolist() == [0, 1]
+
+
 def test_no_agnostic_no_cap_is_plain_topk(orc):
     rng = np.random.default_rng(8)
     for _ in range(50):
