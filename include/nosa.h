@@ -218,6 +218,23 @@ NOSA_API nosa_status nosa_score_select_fetch(nosa_ctx* ctx, const void* q, doubl
                                              int32_t* fetch, int32_t* n_fetch, nosa_stream_t compute,
                                              nosa_stream_t copy);
 
+/* One whole decode step in one call (NOSA summary App. A: select, move the
+ * missed blocks CPU -> GPU, attend): nosa_score_select_fetch followed by
+ * nosa_sparse_decode, with the same results bit for bit.  q (bf16
+ * [B, H_q, d]) and out (bf16 [B, H_q, d]) may each be device memory or pinned
+ * host memory, 16-byte aligned.  Queries in host memory are read over PCIe
+ * once, by the kernel that scores the blocks (up to 512 blocks per unit; with
+ * more, by one copy at the start of the step), and kept in a device copy for
+ * the attention; outputs to host memory are written there directly by the
+ * kernels that finish each unit.  So a decode loop whose queries and outputs
+ * live on the host needs no copies of its own and no wait per step: out is
+ * complete once `compute` has reached the end of the step.
+ * scores, sel, fetch, n_fetch: as in nosa_score_select_fetch (device), or
+ * NULL to use buffers of the context.  Same order rule as
+ * nosa_score_select_fetch (after an optional nosa_append_token). */
+NOSA_API nosa_status nosa_decode_step(nosa_ctx* ctx, const void* q, double* scores, int32_t* sel, int32_t* fetch,
+                                      int32_t* n_fetch, void* out, nosa_stream_t compute, nosa_stream_t copy);
+
 /* Block-sparse GQA attention (NOSA summary App. A): for each query head h of
  * unit u,  out_h = sum_t softmax_t(q_h . K_t / sqrt(d)) V_t  over the tokens of
  * the selected blocks plus the open tail, in fp32 with bf16 inputs; written as

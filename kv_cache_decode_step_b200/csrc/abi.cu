@@ -143,7 +143,15 @@ struct nosa_ctx {
   bool wt_forked = false;
   int wt_grid = 18;
   int prep_warps = 4;       // warps per CTA of the fused score/select/plan kernel
+  // nosa_decode_step: a device copy of queries read from host memory, and the
+  // step buffers used when the caller passes none
+  uint16_t* q_dev = nullptr;
+  double* own_scores = nullptr;
+  int* own_sel = nullptr;
+  int* own_fetch = nullptr;
+  int* own_nfetch = nullptr;
   int attn_stages = 3;      // TMA stages per hits-pass CTA
+  bool attn_producer = true;  // hits pass with a producer warp of its own
 };
 
 namespace {
@@ -227,7 +235,7 @@ void free_all(nosa_ctx* c) {
                   c->slot_block, c->last_used, c->block_slot, c->items, c->n_hit,   c->n_items,
                   c->glist,  c->tail_k,     c->tail_v,    c->a_pending, c->part_o, c->part_ml,
                   c->ds,     c->st,         c->refill_count, c->unit_done, c->done_ctr, c->stage_k,
-                  c->stage_v};
+                  c->stage_v, c->q_dev,  c->own_scores, c->own_sel, c->own_fetch, c->own_nfetch};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (c->ev_plan) cudaEventDestroy(c->ev_plan);
@@ -314,6 +322,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   // attention CTA on its SM, so the grid shrinks to stay in one wave.
   int want = 2 * sms - (c->offloaded ? c->gather_grid : 0);
   if (want < sms) want = sms;
+  if (const char* v = getenv("NOSA_ATTN_PRODUCER")) c->attn_producer = atoi(v) != 0;
   if (const char* v = getenv("NOSA_ATTN_STAGES")) c->attn_stages = atoi(v) == 2 ? 2 : 3;
   if (c->attn_stages == 2) want = 3 * sms - (c->offloaded ? c->gather_grid : 0);
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
@@ -353,6 +362,11 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   ALLOC(c->n_hit, U);
   ALLOC(c->n_items, U);
   ALLOC(c->items, U * K);
+  ALLOC(c->q_dev, (size_t)cfg->batch * cfg->n_q_heads * kD);
+  ALLOC(c->own_scores, U * MB);
+  ALLOC(c->own_sel, U * K);
+  ALLOC(c->own_fetch, U * K);
+  ALLOC(c->own_nfetch, U);
   if (c->offloaded) {
     const size_t CS = c->C;
     ALLOC(c->cache_k, U * CS * kP * kD);
@@ -626,20 +640,13 @@ nosa_status nosa_fetch_missing(nosa_ctx* c, const int32_t* sel, int32_t* fetch, 
   return NOSA_OK;
 }
 
-nosa_status nosa_score_select_fetch(nosa_ctx* c, const void* q, double* scores, int32_t* sel, int32_t* fetch,
-                                    int32_t* n_fetch, nosa_stream_t compute, nosa_stream_t copy) {
-  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
-  if (!c->attached) return fail(NOSA_ERR_ORDER, "score before attach");
-  if (c->phase != kReady) return fail(NOSA_ERR_ORDER, "score must start a step (after decode or append)");
-  if (!q || !scores || !sel || !fetch || !n_fetch)
-    return fail(NOSA_ERR_INVALID, "q, scores, sel, fetch and n_fetch must be non-NULL");
-  if (!prepare_supported(c->max_blocks)) {
-    // beyond the fused kernel's block count: the three calls in a row
-    nosa_status s = nosa_score_blocks(c, q, scores, compute);
-    if (s == NOSA_OK) s = nosa_select(c, scores, sel, compute);
-    if (s == NOSA_OK) s = nosa_fetch_missing(c, sel, fetch, n_fetch, compute, copy);
-    return s;
-  }
+namespace {
+
+// The fused first half of a step.  q_copy: null (q is device memory), or the
+// context's device copy that the kernel fills while it reads q once from
+// (mapped) host memory.
+nosa_status fused_first_half(nosa_ctx* c, const void* q, uint16_t* q_copy, double* scores, int32_t* sel,
+                             int32_t* fetch, int32_t* n_fetch, nosa_stream_t compute, nosa_stream_t copy) {
   nosa_status s = set_device(c);
   if (s != NOSA_OK) return s;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(compute);
@@ -647,6 +654,7 @@ nosa_status nosa_score_select_fetch(nosa_ctx* c, const void* q, double* scores, 
   if ((s = fork_write_through(c, cs)) != NOSA_OK) return s;
   PrepareArgs a{};
   a.sc = score_args(c, q, scores);
+  a.sc.q_copy = q_copy;
   a.se = select_args(c, scores, sel);
   a.pl = plan_args(c, sel, fetch, n_fetch);
   a.offloaded = c->offloaded ? 1 : 0;
@@ -656,6 +664,71 @@ nosa_status nosa_score_select_fetch(nosa_ctx* c, const void* q, double* scores, 
   c->gather_on_side = c->offloaded && xs != cs;
   c->phase = kFetched;
   return NOSA_OK;
+}
+
+}  // namespace
+
+nosa_status nosa_score_select_fetch(nosa_ctx* c, const void* q, double* scores, int32_t* sel, int32_t* fetch,
+                                    int32_t* n_fetch, nosa_stream_t compute, nosa_stream_t copy) {
+  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
+  if (!c->attached) return fail(NOSA_ERR_ORDER, "score before attach");
+  if (c->phase != kReady) return fail(NOSA_ERR_ORDER, "score must start a step (after decode or append)");
+  if (!q || !scores || !sel || !fetch || !n_fetch)
+    return fail(NOSA_ERR_INVALID, "q, scores, sel, fetch and n_fetch must be non-NULL");
+  if (!prepare_supported(c->max_blocks)) {
+    // beyond the fused kernel's block count: scores from the scoring grid,
+    // then selection and plan in one launch (up to 1024 blocks per unit), or
+    // the three calls in a row
+    nosa_status s = nosa_score_blocks(c, q, scores, compute);
+    if (s != NOSA_OK) return s;
+    if (!select_plan_supported(c->max_blocks)) {
+      s = nosa_select(c, scores, sel, compute);
+      if (s == NOSA_OK) s = nosa_fetch_missing(c, sel, fetch, n_fetch, compute, copy);
+      return s;
+    }
+    NOSA_CUDA(launch_select_plan(select_args(c, scores, sel), plan_args(c, sel, fetch, n_fetch), c->offloaded ? 1 : 0,
+                                 reinterpret_cast<cudaStream_t>(compute)));
+    c->copy_stream = reinterpret_cast<cudaStream_t>(copy);
+    c->gather_on_side = c->offloaded && copy != compute;
+    c->phase = kFetched;
+    return NOSA_OK;
+  }
+  return fused_first_half(c, q, nullptr, scores, sel, fetch, n_fetch, compute, copy);
+}
+
+nosa_status nosa_decode_step(nosa_ctx* c, const void* q, double* scores, int32_t* sel, int32_t* fetch,
+                             int32_t* n_fetch, void* out, nosa_stream_t compute, nosa_stream_t copy) {
+  if (!c) return fail(NOSA_ERR_INVALID, "ctx is NULL");
+  if (!c->attached) return fail(NOSA_ERR_ORDER, "step before attach");
+  if (c->phase != kReady) return fail(NOSA_ERR_ORDER, "a step starts after decode or append");
+  if (!q || !out) return fail(NOSA_ERR_INVALID, "q and out must be non-NULL");
+  nosa_status s = set_device(c);
+  if (s != NOSA_OK) return s;
+  void *qd = nullptr, *od = nullptr;
+  const int qk = pointer_kind(q, &qd), ok = pointer_kind(out, &od);
+  if (qk == 0 || ok == 0) return fail(NOSA_ERR_INVALID, "q and out must be device or pinned host memory");
+  if ((reinterpret_cast<uintptr_t>(qd) | reinterpret_cast<uintptr_t>(od)) % 16 != 0)
+    return fail(NOSA_ERR_INVALID, "q and out must be 16-byte aligned");
+  if (!scores) scores = c->own_scores;
+  if (!sel) sel = c->own_sel;
+  if (!fetch) fetch = c->own_fetch;
+  if (!n_fetch) n_fetch = c->own_nfetch;
+  const void* q_attn = qd;  // the queries the attention reads: device memory
+  if (qk == 2) {
+    q_attn = c->q_dev;
+    if (prepare_supported(c->max_blocks)) {
+      s = fused_first_half(c, qd, c->q_dev, scores, sel, fetch, n_fetch, compute, copy);
+    } else {
+      // beyond the fused kernel's block count: one copy in, then the three calls
+      NOSA_CUDA(cudaMemcpyAsync(c->q_dev, q, (size_t)c->cfg.batch * c->cfg.n_q_heads * kD * 2,
+                                cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(compute)));
+      s = nosa_score_select_fetch(c, c->q_dev, scores, sel, fetch, n_fetch, compute, copy);
+    }
+  } else {
+    s = nosa_score_select_fetch(c, qd, scores, sel, fetch, n_fetch, compute, copy);
+  }
+  if (s != NOSA_OK) return s;
+  return nosa_sparse_decode(c, q_attn, sel, od, compute);
 }
 
 nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, void* out, nosa_stream_t stream) {
@@ -726,7 +799,7 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
   }
   // hits pass: blocks already on the GPU (all of S(t) when KV is in HBM) plus
   // the open tail
-  NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st, c->attn_stages));
+  NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st, c->attn_stages, c->attn_producer));
   if (c->gather_on_side) NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
   if (c->appends_enabled) {
     CloseArgs cl{};

@@ -24,6 +24,8 @@ constexpr int kStageBytes = 2 * kBlockBytes;
 // Shared memory of a CTA with S stages: the stages, S mbarriers, a flag word
 // and slack for 1024-byte alignment.
 constexpr int smem_bytes_for(int S) { return S * kStageBytes + S * 8 + 16 + 1024; }
+// The producer-warp pass: S FULL and S EMPTY mbarriers.
+constexpr int smem_ws_bytes_for(int S) { return S * kStageBytes + 2 * S * 8 + 16 + 1024; }
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 // Issue the TMA loads of one block (K and V: four 64 x 64 boxes, 32 KiB).
@@ -172,6 +174,142 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   }
 }
 
+// The same pass with a producer warp of its own.  Warp 4 (one thread) walks
+// the CTA's positions and keeps kStages blocks of TMA loads in flight, each
+// stage guarded by a FULL mbarrier (the loads' bytes) and an EMPTY one (the
+// four consumer warps); warps 0-3 attend the blocks in the same order.  A
+// segment's end (its partial, the unit count, the next unit's queries) no
+// longer holds up the loads: only the stage that the partial is staged
+// through stays busy until it is written.  Positions are tracked as
+// (unit, index) pairs instead of being divided out of a flat index, and a
+// segment's last valid position is known in closed form.  Same walk, same
+// partials, same arithmetic: the outputs are bit-identical to the pass above.
+constexpr int kBarCons = 1;  // named barrier: the consumer warps alone
+
+template <int kStages>
+__global__ void __launch_bounds__(kAttnThreads + 32, 2)
+    attend_hits_ws_kernel(const __grid_constant__ DecodeMaps maps, DecodeArgs a) {
+  extern __shared__ unsigned char attn_smem_raw[];
+  unsigned char* sm = aligned_smem(attn_smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  int* s_flag = reinterpret_cast<int*>(empty + kStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tail_len = a.tail_split ? a.ds->tail_len_step : 0;
+  Walk wk;
+  wk.vpu = a.vpu;
+  wk.V = (long long)a.U * wk.vpu;
+  wk.grid = gridDim.x;
+  const long long p0 = wk.start(blockIdx.x), p1 = wk.start(blockIdx.x + 1);
+  const int vpu = a.vpu;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);  // one arrival per consumer warp
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (p0 >= p1) return;
+  const int u0 = (int)(p0 / vpu), j0 = (int)(p0 % vpu);
+  const int npos = (int)(p1 - p0);
+
+  if (warp == 4) {
+    // ---- producer
+    if (lane != 0) return;
+    int u = u0, j = j0, issued = 0;
+    int n_hit_u = a.resident ? a.k : a.n_hit[u];
+    bool timed_out = false;
+    for (int q = 0; q < npos; ++q) {
+      if (position_valid(a, j, n_hit_u, tail_len)) {
+        const int st = issued % kStages;
+        if (issued >= kStages &&
+            !mbar_wait_bounded(&empty[st], (uint32_t)((issued / kStages - 1) & 1), kWaitLimitNs)) {
+          timed_out = true;
+          break;
+        }
+        // the consumers' reads of this stage come before the copies into it
+        fence_proxy_async_smem();
+        issue_block(maps, a, sm, full, st, u, j < a.k ? j : 0, j >= a.k);
+        ++issued;
+      }
+      if (++j == vpu) {
+        j = 0;
+        ++u;
+        if (q + 1 < npos) n_hit_u = a.resident ? a.k : a.n_hit[u];
+      }
+    }
+    if (timed_out) atomicOr(&a.ds->error_bits, ERR_TIMEOUT);
+    // every stage's last loads land before this thread leaves
+    for (int g2 = issued - 1; g2 >= 0 && g2 >= issued - kStages; --g2)
+      (void)mbar_wait_bounded(&full[g2 % kStages], (uint32_t)((g2 / kStages) & 1), kWaitLimitNs);
+    return;
+  }
+
+  // ---- consumers
+  const auto cons_sync = [] { bar_sync(kBarCons, kAttnThreads); };
+  int gb = 0;  // blocks consumed
+  int u = u0, j = j0, q = 0;
+  while (q < npos) {
+    // one segment: the positions of unit u inside this CTA's range
+    const int seg_len = min(npos - q, vpu - j);
+    const int n_hit_u = a.resident ? a.k : a.n_hit[u];
+    const int first_cta = wk.cta_of((long long)u * vpu);
+    const int n_segs = wk.cta_of((long long)(u + 1) * vpu - 1) - first_cta + 1;
+    const size_t part = (size_t)u * a.nparts + a.part_base + (blockIdx.x - first_cta);
+    float* po = a.part_o + part * a.G * kD;
+    float2* pml = a.part_ml + part * a.G;
+    // the segment's last valid position (-1: none): the open tail if the
+    // segment reaches it, else its last block in [j, j + seg_len)
+    const int seg_end = j + seg_len - 1;
+    int seg_last;
+    if (tail_len > 0 && seg_end >= a.k && j <= a.k) {
+      seg_last = a.k;
+    } else {
+      seg_last = min(seg_end, (a.resident ? a.k : n_hit_u) - 1);
+      if (seg_last < j) seg_last = -1;
+    }
+
+    uint32_t qf[8][2];
+    load_query(a, u, lane, qf);
+    AttnAcc acc;
+    acc_init(acc);
+    int consumed_here = 0;
+    for (int jj = j; jj < j + seg_len; ++jj) {
+      if (!position_valid(a, jj, n_hit_u, tail_len)) continue;
+      const int st = gb % kStages;
+      const bool ok = mbar_wait_bounded(&full[st], (uint32_t)((gb / kStages) & 1), kWaitLimitNs);
+      if (bar_red_or(kBarCons, kAttnThreads, !ok)) {
+        if (threadIdx.x == 0) atomicOr(&a.ds->error_bits, ERR_TIMEOUT);
+        return;
+      }
+      const uint32_t kb = smem_u32(sm + st * kStageBytes);
+      attend_block(kb, kb + kBlockBytes, warp, lane, jj < a.k ? kP : tail_len, qf, acc);
+      ++gb;
+      ++consumed_here;
+      if (jj == seg_last) {
+        // the segment's partial, merged through the stage just consumed
+        cons_sync();  // every consumer warp is done reading the stage
+        const WarpStates ws(sm + st * kStageBytes);
+        publish_warp_state(acc, ws, warp, lane, cons_sync);
+        store_partial(ws, a.G, po, pml, threadIdx.x, kAttnThreads);
+        cons_sync();
+      } else {
+        __syncwarp();
+      }
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    if (consumed_here == 0 && threadIdx.x < a.G) pml[threadIdx.x] = make_float2(-INFINITY, 0.f);
+
+    // whoever completes the unit's partials (this CTA, another segment's, or
+    // the gather of its last fetched block) merges them
+    contribute_partial(a, u, n_segs, fetched_blocks(a, u), threadIdx.x, kAttnThreads, s_flag, cons_sync);
+    q += seg_len;
+    j = 0;
+    ++u;
+  }
+}
+
 // Partial slots a unit needs in the hits pass for a grid of `grid` CTAs.
 __host__ __device__ inline int hits_segments_per_unit(int U, int vpu, int grid) {
   // a unit spans at most ceil(vpu * grid / V) + 1 CTA ranges, V = U * vpu
@@ -186,11 +324,27 @@ cudaError_t configure_decode() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attend_hits_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes_for(2));
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attend_hits_ws_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_ws_bytes_for(3));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attend_hits_ws_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_ws_bytes_for(2));
+  if (e != cudaSuccess) return e;
+
   return configure_gather_attend();
 }
 
 // stages: TMA stages per CTA (2 or 3); the grid's CTAs per SM follow from it.
-cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st, int stages) {
+cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st, int stages,
+                               bool producer_warp) {
+  if (producer_warp) {
+    if (stages == 2) {
+      attend_hits_ws_kernel<2><<<grid, kAttnThreads + 32, smem_ws_bytes_for(2), st>>>(m, a);
+    } else {
+      attend_hits_ws_kernel<3><<<grid, kAttnThreads + 32, smem_ws_bytes_for(3), st>>>(m, a);
+    }
+    return cudaGetLastError();
+  }
   if (stages == 2) {
     attend_hits_kernel<2><<<grid, kAttnThreads, smem_bytes_for(2), st>>>(m, a);
   } else {

@@ -116,6 +116,24 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// Untiled bulk copy shared -> global in this thread's bulk async-group,
+// committed; wait_read: this thread's groups have read their shared memory;
+// wait_all: and completed.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(gdst)),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Plain arrival on an mbarrier (no transaction bytes).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -218,7 +236,9 @@ cudaError_t launch_pool(const uint16_t* src, size_t src_unit_tokens, int U, int 
                         uint16_t* kbar, int kbar_unit_rows, cudaStream_t st);
 
 struct ScoreArgs {
-  const uint16_t* q;        // [B, Hq, d]
+  const uint16_t* q;        // [B, Hq, d]; device memory, or mapped pinned host memory when q_copy is set
+  uint16_t* q_copy;         // null, or [B, Hq, d] device: the fused kernel reads each unit's queries once
+                            // (staged in shared memory) and leaves a device copy here for the attention
   const uint16_t* kbar;     // [U, max_blocks*R, d]
   double* scores;           // [U, max_blocks]
   DevState* ds;
@@ -270,6 +290,10 @@ struct PrepareArgs {
 };
 bool prepare_supported(int max_blocks);
 cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t st);
+// Selection and plan in one launch (one warp per unit), after score_kernel;
+// for max_blocks <= 1024.  Same results as launch_select then launch_plan.
+bool select_plan_supported(int max_blocks);
+cudaError_t launch_select_plan(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st);
 
 struct GatherArgs {
   const uint16_t* hk;       // host K (device-addressable), [U, max_blocks*P, d]
@@ -312,8 +336,9 @@ struct DecodeMaps {
 };
 // Hits pass (persistent, `grid` CTAs, which must equal a.hits_grid); partials,
 // and with unit_done the output.
+// producer_warp: the variant with a producer warp of its own (same results).
 cudaError_t launch_attend_hits(const DecodeArgs& a, const DecodeMaps& m, int grid, cudaStream_t st,
-                               int stages = 3);
+                               int stages = 3, bool producer_warp = true);
 // The hits-pass grid for a requested CTA count (at most one CTA per position).
 int attend_hits_grid(int U, int vpu, int want);
 // Partial slots per unit the hits pass writes for this shape and requested grid.
@@ -340,6 +365,19 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
 }
 __device__ __forceinline__ void bar_arrive(int id, int count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier over `count` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool bar_red_or(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 struct AppendArgs {

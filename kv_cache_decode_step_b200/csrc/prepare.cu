@@ -18,7 +18,8 @@ namespace nosa {
 
 constexpr int kPrepMaxThreads = 512;
 
-// Shared memory: scores [max_blocks] fp64, selection bitmaps [2][R] words,
+// Shared memory: the unit's query rows [G][16] uint4 (staged when they are
+// read from host memory), scores [max_blocks] fp64, selection bitmaps [2][R] words,
 // plan scratch (max(32, 2C + 2k) ints), then copies of the unit's S(t-1) [k],
 // Gamma_e(t-1) [k_e], the new selection [k], the register plan's slot tables
 // [32] x 2 and the general plan's block -> slot table [max_blocks].  The
@@ -28,7 +29,8 @@ template <int R>
 __global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs a) {
   extern __shared__ __align__(16) unsigned char prep_smem[];
   const int k = a.se.k, ke = a.se.k_e, C = a.pl.C;
-  double* ssc = reinterpret_cast<double*>(prep_smem);
+  uint4* s_q = reinterpret_cast<uint4*>(prep_smem);  // the unit's query rows when they are staged
+  double* ssc = reinterpret_cast<double*>(s_q + kMaxG * kRowU4);
   unsigned(*sbm)[R] = reinterpret_cast<unsigned(*)[R]>(ssc + a.sc.max_blocks);
   int* psm = reinterpret_cast<int*>(sbm + 2);
   int* s_prev = psm + a.plan_ints;
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs
       cp_async4(s_bs + i, a.pl.block_slot + (size_t)u * a.pl.max_blocks + i);
   }
 
-  score_unit_warps(a.sc, u, warp, blockDim.x >> 5, lane, ssc);
+  score_unit_warps(a.sc, u, warp, blockDim.x >> 5, lane, ssc, s_q);
   cp_async_wait_all();
   __syncthreads();
   if (warp != 0) return;
@@ -83,7 +85,8 @@ __global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs
 template <int R>
 cudaError_t launch_prepare_r(PrepareArgs a, cudaStream_t st) {
   a.plan_ints = a.offloaded ? max(32, 2 * a.pl.C + 2 * a.pl.k) : 0;
-  const size_t smem = (size_t)a.sc.max_blocks * sizeof(double) + 2 * R * sizeof(unsigned) +
+  const size_t smem = kMaxG * kRowU4 * sizeof(uint4) + (size_t)a.sc.max_blocks * sizeof(double) +
+                      2 * R * sizeof(unsigned) +
                       (size_t)(a.plan_ints + 2 * a.se.k + a.se.k_e + 64) * sizeof(int) +
                       (a.offloaded ? (size_t)a.pl.max_blocks * sizeof(int) : 0);
   if (smem > 48 * 1024) {
@@ -96,6 +99,61 @@ cudaError_t launch_prepare_r(PrepareArgs a, cudaStream_t st) {
 }
 
 bool prepare_supported(int max_blocks) { return max_blocks <= kPrepareMaxBlocks; }
+
+// Beyond kPrepareMaxBlocks the scores come from score_kernel (many CTAs per
+// unit); selection and plan then still run as one launch: one warp per unit
+// selects (register path, up to 1024 blocks) and plans from a copy of the
+// selection in shared memory.  Shared memory per warp: the selection [k] and
+// the general plan's scratch (2C + 2k ints).
+constexpr int kSelPlanWarps = 4;
+
+template <int R>
+__global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectArgs se, PlanArgs pl, int offloaded,
+                                                                        int plan_ints) {
+  extern __shared__ __align__(16) int sp_smem[];
+  __shared__ unsigned sbm[kSelPlanWarps][2][R];
+  __shared__ int ssrc[kSelPlanWarps][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * kSelPlanWarps + warp;
+  // the gather that follows claims its entries from 0
+  if (blockIdx.x == 0 && threadIdx.x == 0) se.ds->gather_next = 0;
+  if (u >= se.U) return;
+  int* s_sel = sp_smem + (size_t)warp * (se.k + plan_ints);
+  select_unit_reg<R>(se, u, lane, sbm[warp], se.scores + (size_t)u * se.max_blocks, se.prev + (size_t)u * se.k,
+                     se.ge + (size_t)u * se.k_e, s_sel);
+  __syncwarp();  // the selection is read back by the plan
+  if (!offloaded) {
+    for (int i = lane; i < se.k; i += 32) pl.fetch[(size_t)u * se.k + i] = -1;
+    if (lane == 0) pl.n_fetch[u] = 0;
+  } else if (pl.C <= 32 && pl.k <= 32) {
+    plan_unit_reg(pl, u, lane, ssrc[warp], s_sel, pl.slot_block + (size_t)u * pl.C, pl.last_used + (size_t)u * pl.C);
+  } else {
+    plan_unit_smem(pl, u, lane, s_sel + se.k, s_sel, pl.block_slot + (size_t)u * pl.max_blocks, false);
+  }
+}
+
+template <int R>
+cudaError_t launch_select_plan_r(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st) {
+  const int plan_ints = offloaded ? 2 * pl.C + 2 * pl.k : 0;
+  const size_t smem = (size_t)kSelPlanWarps * (se.k + plan_ints) * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e =
+        cudaFuncSetAttribute(select_plan_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  const int grid = (se.U + kSelPlanWarps - 1) / kSelPlanWarps;
+  select_plan_kernel<R><<<grid, kSelPlanWarps * 32, smem, st>>>(se, pl, offloaded, plan_ints);
+  return cudaGetLastError();
+}
+
+bool select_plan_supported(int max_blocks) { return max_blocks <= 1024; }
+
+cudaError_t launch_select_plan(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st) {
+  const int rows = (se.max_blocks + 31) / 32;
+  if (rows <= 16) return launch_select_plan_r<16>(se, pl, offloaded, st);
+  if (rows <= 32) return launch_select_plan_r<32>(se, pl, offloaded, st);
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t st) {
   const int rows = (a.sc.max_blocks + 31) / 32;

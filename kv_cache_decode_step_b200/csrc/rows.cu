@@ -88,15 +88,6 @@ constexpr int kBulkSmemBytes = 1024 + kBulkWarps * kBulkRingBytes;
 constexpr int kBulkPieceMax = 16384;
 constexpr uint64_t kBulkWaitNs = 1000000000ull;
 
-__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(gdst)),
-               "r"(smem_u32(ssrc)), "r"(bytes)
-               : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // a.total counts pieces here, log_piece = log2(piece bytes), a.log_cpr =
 // log2(pieces per row); nslots = min(kBulkSlots, kBulkRingBytes / piece).
@@ -150,6 +141,7 @@ __global__ void __launch_bounds__(kBulkThreads) gather_rows_bulk_kernel(RowsArgs
       break;
     }
     bulk_store(dst + dst_off[slot], ring + (size_t)slot * piece, piece);
+    bulk_commit();
     ++tail;
     // the slot of the piece just stored is reloaded once the store has read it
     bulk_wait_read_all();

@@ -32,7 +32,7 @@ ENTRY_POINTS = (
     "nosa_check_errors", "nosa_read_cache_map", "nosa_get_state", "nosa_set_state",
     "nosa_debug_wait_flag", "nosa_last_error", "nosa_version", "nosa_sparse_decode_noalloc",
     "nosa_gather_rows", "nosa_score_select_fetch", "nosa_gather_rows_bulk", "nosa_noalloc_check_errors",
-    "nosa_read_cache", "nosa_debug_inject_cuda_error",
+    "nosa_read_cache", "nosa_debug_inject_cuda_error", "nosa_decode_step",
 )
 
 
@@ -99,6 +99,7 @@ def lib() -> C.CDLL:
             "nosa_gather_rows": ([vp, C.c_int64, vp, C.c_int64, i32, vp, vp, i32, i32, vp, vp], st),
             "nosa_gather_rows_bulk": ([vp, C.c_int64, vp, C.c_int64, i32, vp, vp, i32, i32, vp, vp], st),
             "nosa_score_select_fetch": ([vp, vp, vp, vp, vp, vp, vp, vp], st),
+            "nosa_decode_step": ([vp, vp, vp, vp, vp, vp, vp, vp, vp], st),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -183,6 +184,13 @@ def nosa_score_select_fetch(ctx, q, scores, sel, fetch, n_fetch, compute=None, c
     _check(lib().nosa_score_select_fetch(ctx, _ptr(q), _ptr(scores), _ptr(sel), _ptr(fetch), _ptr(n_fetch),
                                          _stream(compute), _stream(copy if copy is not None else compute)),
            "nosa_score_select_fetch")
+
+
+def nosa_decode_step(ctx, q, out, scores=None, sel=None, fetch=None, n_fetch=None, compute=None,
+                     copy=None) -> None:
+    _check(lib().nosa_decode_step(ctx, _ptr(q), _ptr(scores), _ptr(sel), _ptr(fetch), _ptr(n_fetch), _ptr(out),
+                                  _stream(compute), _stream(copy if copy is not None else compute)),
+           "nosa_decode_step")
 
 
 def nosa_sparse_decode(ctx, q, sel, out, stream=None) -> None:

@@ -129,6 +129,23 @@ class Decoder:
             nosa.nosa_fetch_missing(self.ctx, self.sel, self.fetch, self.n_fetch, s, cs)
         nosa.nosa_sparse_decode(self.ctx, self.q, self.sel, self.out, s)
 
+    def step_through(self, q, out) -> None:
+        """Eager step t through nosa_decode_step: q and out may be device or
+        pinned host tensors [B, H_q, d] bf16 (the library reads and writes
+        them itself).  For growing sequences the appended token's K/V (and
+        agnostic score) are copied into the static append buffers first."""
+        t = self.t
+        s = self.stream
+        with torch.cuda.stream(s):
+            if self.w.append:
+                self.k_in.copy_(self.k_new[t], non_blocking=True)
+                self.v_in.copy_(self.v_new[t], non_blocking=True)
+                self.a_in.copy_(self.a_new[t], non_blocking=True)
+                nosa.nosa_append_token(self.ctx, self.k_in, self.v_in, self.a_in, s)
+            nosa.nosa_decode_step(self.ctx, q, out, self.scores, self.sel, self.fetch, self.n_fetch, s,
+                                  self.copy_stream)
+        self.t += 1
+
     def step(self) -> None:
         """Eager step t (queries of step t copied into the static q buffer)."""
         t = self.t

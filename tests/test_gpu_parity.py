@@ -163,6 +163,26 @@ def test_two_stage_hits_pass(offloaded, monkeypatch):
     _full(w, range(w.units), range(w.steps), cache_steps=[w.steps - 1] if offloaded else ())
 
 
+@pytest.mark.parametrize("offloaded", [True, False])
+def test_hits_pass_without_a_producer_warp(offloaded, monkeypatch):
+    """The hits pass whose thread 0 issues the loads between blocks
+    (NOSA_ATTN_PRODUCER=0) gives the same outputs as the default pass with a
+    producer warp, bit for bit."""
+    w = configs.get("layer8b", batch=2, steps=10)
+    if offloaded:
+        w = w.with_(offloaded=True, cache_factor=2)
+    data = inputs.generate(w)
+    sample = list(range(w.units))
+    a = run_gpu(w, data, sample, range(w.steps))
+    monkeypatch.setenv("NOSA_ATTN_PRODUCER", "0")
+    b = run_gpu(w, data, sample, range(w.steps))
+    assert np.array_equal(a.sel, b.sel) and np.array_equal(a.fetch, b.fetch)
+    for t in a.out:
+        assert np.array_equal(a.out[t], b.out[t]), t
+    refs = run_oracle(w, data, sample, range(w.steps))
+    compare(w, b, refs, sample)
+
+
 @pytest.mark.parametrize("gap", [0, 17])
 @pytest.mark.parametrize("offloaded", [True, False])
 def test_hits_pass_walk_gap(gap, offloaded, monkeypatch):
