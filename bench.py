@@ -431,7 +431,7 @@ def run_ours(args):
                  "unit": "GB/s", "frac": gather_gbs / h2d_peak if h2d_peak else None, "traffic": None,
                  "peak_source": "pinned cudaMemcpyAsync H2D measured in this run (256 MiB)",
                  "bytes_per_launch": phase["fetched_bytes_per_step"], "ms_per_launch": gather_ms}
-    rl_attn = {"kernel": "attend_hits_kernel", "bound": "hbm", "achieved": attn_gbs,
+    rl_attn = {"kernel": "attend_hits_ws_kernel", "bound": "hbm", "achieved": attn_gbs,
                "peak": hbm_meas, "unit": "GB/s", "frac": attn_gbs / hbm_meas, "traffic": None,
                "peak_source": f"hbm_gbs {hbm_src}", "bytes_per_launch": attn_bytes, "ms_per_launch": attn_ms}
     if w.offloaded:
@@ -573,7 +573,8 @@ APPEND_TIMED_STEPS = 2400  # most timed steps of a growing workload (its KV capa
 # full capture of the dominant kernel on its workload (pcie: link-level read
 # bytes, the traffic that bounds the gather).  Retake after changing the kernel.
 NCU_TRAFFIC = {
-    ("gather_attend_kernel", "offload_b64"): {"dram": 590848 + 29440, "pcie_read": 20717568},
+    ("gather_attend_kernel", "offload_b64"): {"dram": 591616 + 17664, "pcie_read": 20717568},
+    ("attend_hits_ws_kernel", "layer8b"): {"dram": 268951808 + 5076480},
 }
 
 

@@ -103,13 +103,17 @@ bool prepare_supported(int max_blocks) { return max_blocks <= kPrepareMaxBlocks;
 // Beyond kPrepareMaxBlocks the scores come from score_kernel (many CTAs per
 // unit); selection and plan then still run as one launch: one warp per unit
 // selects (register path, up to 1024 blocks) and plans from a copy of the
-// selection in shared memory.  Shared memory per warp: the selection [k] and
-// the general plan's scratch (2C + 2k ints).
+// selection in shared memory.  The unit's slot tables (and, for the general
+// plan, its block -> slot table) arrive in shared memory by cp.async while
+// the selection runs, so the plan reads no global memory of its own.
+// Shared memory per warp (wide_ints): the selection [k], then the general
+// plan's scratch (2C + 2k ints, slot tables first) and block -> slot table
+// [max_blocks], or the register plan's slot tables [32] x 2.
 constexpr int kSelPlanWarps = 4;
 
 template <int R>
 __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectArgs se, PlanArgs pl, int offloaded,
-                                                                        int plan_ints) {
+                                                                        int wide_ints) {
   extern __shared__ __align__(16) int sp_smem[];
   __shared__ unsigned sbm[kSelPlanWarps][2][R];
   __shared__ int ssrc[kSelPlanWarps][32];
@@ -118,31 +122,47 @@ __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectA
   // the gather that follows claims its entries from 0
   if (blockIdx.x == 0 && threadIdx.x == 0) se.ds->gather_next = 0;
   if (u >= se.U) return;
-  int* s_sel = sp_smem + (size_t)warp * (se.k + plan_ints);
+  const int C = pl.C;
+  const bool reg_plan = offloaded && C <= 32 && pl.k <= 32;
+  int* s_sel = sp_smem + (size_t)warp * wide_ints;
+  int* s_plan = s_sel + se.k;                 // general plan: slot tables, then its scratch
+  int* s_bs = s_plan + 2 * C + 2 * pl.k;      // general plan: block -> slot
+  int* s_sb = s_plan;                         // register plan: slot -> block [32]
+  int* s_lu = s_plan + 32;                    //                slot -> last step [32]
+  if (offloaded) {
+    for (int i = lane; i < C; i += 32) {
+      cp_async4(s_sb + i, pl.slot_block + (size_t)u * C + i);
+      cp_async4((reg_plan ? s_lu : s_plan + C) + i, pl.last_used + (size_t)u * C + i);
+    }
+    if (!reg_plan)
+      for (int i = lane; i < pl.max_blocks; i += 32) cp_async4(s_bs + i, pl.block_slot + (size_t)u * pl.max_blocks + i);
+  }
   select_unit_reg<R>(se, u, lane, sbm[warp], se.scores + (size_t)u * se.max_blocks, se.prev + (size_t)u * se.k,
                      se.ge + (size_t)u * se.k_e, s_sel);
-  __syncwarp();  // the selection is read back by the plan
+  cp_async_wait_all();
+  __syncwarp();  // the selection and the tables are read back by the plan
   if (!offloaded) {
     for (int i = lane; i < se.k; i += 32) pl.fetch[(size_t)u * se.k + i] = -1;
     if (lane == 0) pl.n_fetch[u] = 0;
-  } else if (pl.C <= 32 && pl.k <= 32) {
-    plan_unit_reg(pl, u, lane, ssrc[warp], s_sel, pl.slot_block + (size_t)u * pl.C, pl.last_used + (size_t)u * pl.C);
+  } else if (reg_plan) {
+    plan_unit_reg(pl, u, lane, ssrc[warp], s_sel, s_sb, s_lu);
   } else {
-    plan_unit_smem(pl, u, lane, s_sel + se.k, s_sel, pl.block_slot + (size_t)u * pl.max_blocks, false);
+    plan_unit_smem(pl, u, lane, s_plan, s_sel, s_bs, true);
   }
 }
 
 template <int R>
 cudaError_t launch_select_plan_r(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st) {
-  const int plan_ints = offloaded ? 2 * pl.C + 2 * pl.k : 0;
-  const size_t smem = (size_t)kSelPlanWarps * (se.k + plan_ints) * sizeof(int);
+  const bool reg_plan = offloaded && pl.C <= 32 && pl.k <= 32;
+  const int wide_ints = se.k + (!offloaded ? 0 : reg_plan ? 64 : 2 * pl.C + 2 * pl.k + pl.max_blocks);
+  const size_t smem = (size_t)kSelPlanWarps * wide_ints * sizeof(int);
   if (smem > 48 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(select_plan_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   const int grid = (se.U + kSelPlanWarps - 1) / kSelPlanWarps;
-  select_plan_kernel<R><<<grid, kSelPlanWarps * 32, smem, st>>>(se, pl, offloaded, plan_ints);
+  select_plan_kernel<R><<<grid, kSelPlanWarps * 32, smem, st>>>(se, pl, offloaded, wide_ints);
   return cudaGetLastError();
 }
 
