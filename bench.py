@@ -403,7 +403,8 @@ def run_ours(args):
     phase["attention_ms"] = phase1["decode_ms"]
     phase["single_stream_step_ms"] = phase1["step_ms"]
     phase["note"] = ("graph-captured step with timing events between the ABI calls; gather_ms (the fused "
-                     "gather + miss attention, from the end of the plan) from the side-stream pass; "
+                     "gather + miss attention, from the end of the plan to the end of the step, the hits pass "
+                     "running beside it and ending first: hits_side_ms) from the side-stream pass; "
                      "attention_ms = the decode call of a single-stream pass (KV in HBM: the hits pass; KV in "
                      "host memory: the gather + miss attention, then the hits pass)")
 
@@ -445,6 +446,10 @@ def run_ours(args):
         dominant["traffic"] = tr["dram"]
         if "pcie_read" in tr:
             dominant["traffic_pcie_read"] = tr["pcie_read"]
+        if "payload" in tr:
+            # the host-memory bytes the captured launch read (its own misses), beside its link bytes
+            dominant["traffic_payload"] = tr["payload"]
+            dominant["traffic_link_per_payload"] = tr["pcie_read"] / tr["payload"]
         dominant["traffic_source"] = "ncu capture of this kernel on this workload (bytes per launch)"
 
     result = None
@@ -527,15 +532,16 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
             ev["c"].record(s)
             nosa.nosa_fetch_missing(dec.ctx, dec.sel, dec.fetch, dec.n_fetch, s, cs)
         ev["d"].record(s)
-        # the decode call launches the fused gather + miss attention on the copy
-        # stream beside the hits pass: g marks its end
+        # the decode call launches the fused gather + miss attention on s and,
+        # with a second stream, the hits pass beside it on cs: g marks the hits
+        # pass's end, e the gather's (the library joins cs back into s)
         nosa.nosa_sparse_decode(dec.ctx, dec.q, dec.sel, dec.out, s)
         ev["g"].record(cs)
         if cs is not s:
             s.wait_stream(cs)  # join the timing node recorded on the copy stream
         ev["e"].record(s)
     acc = {"score_ms": 0.0, "select_ms": 0.0, "plan_ms": 0.0, "prepare_ms": 0.0, "gather_ms": 0.0,
-           "decode_ms": 0.0, "step_ms": 0.0}
+           "hits_side_ms": 0.0, "decode_ms": 0.0, "step_ms": 0.0}
     fb0 = dec.stats()["fetched_bytes"]
     for _ in range(n):
         t = dec.t
@@ -549,7 +555,8 @@ def instrumented_pass(torch, dec, w, nosa, n, single_stream):
         acc["plan_ms"] += ev["c"].elapsed_time(ev["d"])
         acc["prepare_ms"] += ev["a"].elapsed_time(ev["d"])
         if cs is not s and w.offloaded:
-            acc["gather_ms"] += ev["d"].elapsed_time(ev["g"])
+            acc["gather_ms"] += ev["d"].elapsed_time(ev["e"])
+            acc["hits_side_ms"] += ev["d"].elapsed_time(ev["g"])
         acc["decode_ms"] += ev["d"].elapsed_time(ev["e"])
         acc["step_ms"] += ev["a"].elapsed_time(ev["e"])
     del g
@@ -573,7 +580,8 @@ APPEND_TIMED_STEPS = 2400  # most timed steps of a growing workload (its KV capa
 # full capture of the dominant kernel on its workload (pcie: link-level read
 # bytes, the traffic that bounds the gather).  Retake after changing the kernel.
 NCU_TRAFFIC = {
-    ("gather_attend_kernel", "offload_b64"): {"dram": 591616 + 17664, "pcie_read": 20717568},
+    ("gather_attend_kernel", "offload_b64"): {"dram": 592384 + 36096, "pcie_read": 20717568,
+                                              "payload": 592348 * 32},
     ("attend_hits_ws_kernel", "layer8b"): {"dram": 268951808 + 5076480},
 }
 

@@ -199,9 +199,10 @@ NOSA_API nosa_status nosa_select(nosa_ctx* ctx, const double* scores, int32_t* s
  * (nosa_read_cache_map) are final when it has run.  The copies themselves --
  * K and V of each miss, 2 x 16 KiB, from pinned host memory into its slot by
  * a zero-copy gather kernel that also attends to each block as it lands --
- * are issued by nosa_sparse_decode on `copy`, which may equal compute; a
- * separate copy stream lets the attention to the blocks already cached run
- * beside the transfer.  With KV resident (cache_slots = 0) nothing is copied:
+ * are issued by nosa_sparse_decode on its stream.  `copy` names a second
+ * stream (it may equal compute): when it differs, nosa_sparse_decode runs the
+ * attention to the blocks already cached on it, beside the transfer, and
+ * joins it back.  With KV resident (cache_slots = 0) nothing is copied:
  * fetch is all -1 and n_fetch all 0. */
 NOSA_API nosa_status nosa_fetch_missing(nosa_ctx* ctx, const int32_t* sel, int32_t* fetch,
                                int32_t* n_fetch, nosa_stream_t compute, nosa_stream_t copy);
@@ -240,9 +241,11 @@ NOSA_API nosa_status nosa_decode_step(nosa_ctx* ctx, const void* q, double* scor
  * the selected blocks plus the open tail, in fp32 with bf16 inputs; written as
  * bf16.  q: device bf16 [B, H_q, d]; sel: the same buffer passed to
  * nosa_select; out: device bf16 [B, H_q, d].  With KV in host memory it also
- * issues the miss gather planned by the fetch call, on that call's copy
- * stream (joined back into `stream` before it returns).  Ends the step:
- * closes a full tail block and advances the step counter. */
+ * issues the miss gather planned by the fetch call, on `stream`, and -- when
+ * the fetch call was given a second stream -- runs the attention to the
+ * cached blocks on that stream beside it (joined back into `stream` before
+ * it returns).  Ends the step: closes a full tail block and advances the step
+ * counter. */
 NOSA_API nosa_status nosa_sparse_decode(nosa_ctx* ctx, const void* q, const int32_t* sel, void* out,
                                nosa_stream_t stream);
 

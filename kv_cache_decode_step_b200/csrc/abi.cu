@@ -122,7 +122,7 @@ struct nosa_ctx {
   bool maps_main = false;
   cudaEvent_t ev_plan = nullptr, ev_gather = nullptr;
   bool gather_on_side = false;
-  cudaStream_t copy_stream = nullptr;  // given to the fetch call; the decode call gathers on it
+  cudaStream_t copy_stream = nullptr;  // given to the fetch call; the decode call runs the hits pass on it
 
   // host mirror of the device step state (validation only)
   int h_n_closed = 0, h_tail = 0;
@@ -789,18 +789,22 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
     ga.g.max_blocks = c->max_blocks;
     ga.d = a;
     if (c->gather_on_side) {
+      // the gather goes first, on this stream, so its CTAs are placed before
+      // the hits pass's; the hits pass runs beside it on the second stream
       NOSA_CUDA(cudaEventRecord(c->ev_plan, st));
+      NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, st));
       NOSA_CUDA(cudaStreamWaitEvent(c->copy_stream, c->ev_plan, 0));
-      NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, c->copy_stream));
+      NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, c->copy_stream, c->attn_stages, c->attn_producer));
       NOSA_CUDA(cudaEventRecord(c->ev_gather, c->copy_stream));
+      NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
     } else {
       NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, st));
     }
   }
   // hits pass: blocks already on the GPU (all of S(t) when KV is in HBM) plus
   // the open tail
-  NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st, c->attn_stages, c->attn_producer));
-  if (c->gather_on_side) NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
+  if (!c->gather_on_side)
+    NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, st, c->attn_stages, c->attn_producer));
   if (c->appends_enabled) {
     CloseArgs cl{};
     cl.tail_k = c->tail_k;

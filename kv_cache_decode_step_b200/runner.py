@@ -77,9 +77,10 @@ class Decoder:
         self.n_fetch = torch.zeros((U,), dtype=torch.int32, device=self.dev)
         self.out = torch.zeros((w.batch, w.n_q_heads, d), dtype=torch.bfloat16, device=self.dev)
         self.stream = torch.cuda.Stream(self.dev)
-        # the gather runs on a high-priority side stream so it overlaps attention
-        self.copy_stream = (torch.cuda.Stream(self.dev, priority=-1) if (side_copy_stream and w.offloaded)
-                            else self.stream)
+        # a second stream: the attention to the cached blocks runs on it beside
+        # the miss gather (which the library launches with the highest CTA
+        # priority on the main stream)
+        self.copy_stream = (torch.cuda.Stream(self.dev) if (side_copy_stream and w.offloaded) else self.stream)
         self.ctx = nosa.nosa_create(nosa.config_from_workload(w))
         self.graph: Optional[torch.cuda.CUDAGraph] = None
         self.t = 0
