@@ -53,7 +53,7 @@ def parse():
     p.add_argument("--k-query", type=int, default=None,
                    help="query-aware blocks of the 64-block budget (paper policy; default 16)")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--e2e-steps", type=int, default=2000)
+    p.add_argument("--e2e-steps", type=int, default=500)
     return p.parse_args()
 
 
@@ -316,13 +316,22 @@ def run_ours(args):
     build.build()
 
     base = configs.with_policy(configs.get(args.workload), args.policy, args.k_query)
-    # Queries of a fixed-length workload are reused cyclically past its last
-    # step; a growing workload needs one appended token per step, so its inputs
-    # (and KV capacity) cover every step this run makes, the timed ones capped.
-    timed_cap = max(args.steps, APPEND_TIMED_STEPS) if base.append else None
-    total = (1 + args.warmup + 1 + 32 + WARM_STEPS + (timed_cap or 0) + 2 * min(args.steps, 50)
-             + 2 * (args.e2e_steps + 4) + LATENCY_STEPS + 8)
-    w = base.with_(steps=max(base.steps, total)) if base.append else base
+    # With KV in host memory every step of the run gets a fresh query of the
+    # seeded AR(1) stream: revisiting queries would find their blocks still in
+    # the cache and understate the misses.  The timed steps are capped so the
+    # queries fit a memory budget (growing sequences: their KV capacity).
+    # With KV in HBM there is no cache state, and queries are reused past the
+    # workload's last step.
+    untimed = (1 + args.warmup + 1 + 32 + WARM_STEPS + 2 * min(args.steps, 50) + 2 * (args.e2e_steps + 4)
+               + LATENCY_STEPS + 8)
+    q_step_bytes = base.batch * base.n_q_heads * base.head_dim * 2
+    if base.append:
+        timed_cap = max(args.steps, APPEND_TIMED_STEPS)
+    elif base.offloaded:
+        timed_cap = max(args.steps, min(MAX_QUERY_STEPS, int(QUERY_BUDGET_BYTES // q_step_bytes)) - untimed)
+    else:
+        timed_cap = None
+    w = base.with_(steps=max(base.steps, untimed + timed_cap)) if timed_cap is not None else base
     data = inputs.generate(w)
     dec = runner.Decoder(w, data, device=local)
 
@@ -575,6 +584,8 @@ LATENCY_STEPS = 256
 MIN_TIMED_MS = 1000.0      # the timed region repeats its K steps until this much GPU time has passed
 WARM_STEPS = 64            # untimed replays right before the timed region
 APPEND_TIMED_STEPS = 2400  # most timed steps of a growing workload (its KV capacity is sized for them)
+QUERY_BUDGET_BYTES = 3.5e9  # queries of an offloaded run (on the device, and pinned for the end-to-end pass)
+MAX_QUERY_STEPS = 16000
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu --set
 # full capture of the dominant kernel on its workload (pcie: link-level read
@@ -621,11 +632,10 @@ def e2e_pass(torch, dec, w, nosa, n, host_wait=False, dist=None, world=1, dev=No
     sequences first copy the new token's K/V in and append it.  host_wait:
     also wait on the host for each step's output (a sampling loop)."""
     q_host = dec.q_all.cpu().pin_memory()
-    nq = q_host.shape[0]
     out_host = [torch.empty(dec.out.shape, dtype=dec.out.dtype, pin_memory=True) for _ in range(2)]
     s = dec.stream
     for i in range(4):  # untimed
-        dec.step_through(q_host[dec.t % nq], out_host[i % 2])
+        dec.step_through(q_host[dec.q_index(dec.t)], out_host[i % 2])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     if world > 1:
@@ -633,7 +643,7 @@ def e2e_pass(torch, dec, w, nosa, n, host_wait=False, dist=None, world=1, dev=No
     e0.record(s)
     t0 = time.perf_counter()
     for i in range(n):
-        dec.step_through(q_host[dec.t % nq], out_host[i % 2])
+        dec.step_through(q_host[dec.q_index(dec.t)], out_host[i % 2])
         if host_wait:
             s.synchronize()
     e1.record(s)

@@ -250,6 +250,9 @@ __global__ void __launch_bounds__(kAttnThreads + 32, 2)
   const auto cons_sync = [] { bar_sync(kBarCons, kAttnThreads); };
   int gb = 0;  // blocks consumed
   int u = u0, j = j0, q = 0;
+  // the next segment's queries are loaded while this one streams its blocks
+  uint32_t qf[8][2], qn[8][2];
+  load_query(a, u, lane, qn);
   while (q < npos) {
     // one segment: the positions of unit u inside this CTA's range
     const int seg_len = min(npos - q, vpu - j);
@@ -270,8 +273,12 @@ __global__ void __launch_bounds__(kAttnThreads + 32, 2)
       if (seg_last < j) seg_last = -1;
     }
 
-    uint32_t qf[8][2];
-    load_query(a, u, lane, qf);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qf[ks][0] = qn[ks][0];
+      qf[ks][1] = qn[ks][1];
+    }
+    if (q + seg_len < npos) load_query(a, u + 1, lane, qn);
     AttnAcc acc;
     acc_init(acc);
     int consumed_here = 0;

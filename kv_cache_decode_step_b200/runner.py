@@ -108,11 +108,22 @@ class Decoder:
             pass
 
     # ------------------------------------------------------------ one step
+    def q_index(self, t: int) -> int:
+        """Row of q_all used at step t.  Past the workload's last step the
+        query sequence is walked back and forth (0..N-1, N-2..0, 1..), so
+        consecutive steps always get neighbouring states of the AR(1)
+        sequence instead of jumping from the last query to the first."""
+        n = self.q_all.shape[0]
+        if t < n or n < 2:
+            return t % n
+        p = t % (2 * n - 2)
+        return p if p < n else 2 * n - 2 - p
+
     def _load_inputs(self, t: int) -> None:
         """Copy step t's inputs into the static buffers (on self.stream).
-        Queries are reused cyclically past the workload's last step (a run
-        longer than the workload); appended tokens are not."""
-        self.q.copy_(self.q_all[t % self.q_all.shape[0]], non_blocking=True)
+        Queries are reused past the workload's last step (see q_index);
+        appended tokens are not."""
+        self.q.copy_(self.q_all[self.q_index(t)], non_blocking=True)
         if self.w.append:
             self.k_in.copy_(self.k_new[t], non_blocking=True)
             self.v_in.copy_(self.v_new[t], non_blocking=True)
