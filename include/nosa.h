@@ -17,8 +17,9 @@
  *                       blocks (App. A)
  *
  * plus nosa_append_token first when the sequence grows during decoding.
- * nosa_score_select_fetch makes the first three calls in one (fused below
- * 512 blocks per unit).
+ * nosa_score_select_fetch makes the first three calls in one (one kernel up
+ * to 512 blocks per unit), and nosa_decode_step the whole step, with queries
+ * and outputs in device or pinned host memory.
  *
  * Terms.  A unit is one (sequence b, KV head g), numbered u = b*n_kv_heads + g.
  * G = n_q_heads / n_kv_heads query heads share a KV head; query head h uses KV

@@ -2,11 +2,11 @@
 // zero-copy miss gather.
 //
 // NOSA: Native and Offloadable Sparse Attention (paperlayer summary):
-//   §4     a set-difference kernel between old and new selections builds a
-//          replacement mapping; only blocks unused by the current step are
-//          swapped out, since GPU-resident blocks need not be contiguous; a
-//          transfer kernel reads fine-grained 16 KiB blocks through unified
-//          virtual addressing;
+//   §4     the old and new selections are compared by a dedicated kernel
+//          that decides which cached blocks give up their slots; a block
+//          the step still needs keeps its slot, and slots need not be
+//          contiguous; a transfer kernel reads 16 KiB blocks from host memory
+//          through unified virtual addressing;
 //   App. A per step, the cache-missed blocks move CPU -> GPU.
 // Replacement order: free slots (lowest first), then resident blocks outside
 // S(t) by (last step selected, block id) ascending.  The i-th miss (ascending

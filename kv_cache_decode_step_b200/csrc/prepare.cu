@@ -2,7 +2,7 @@
 // kernel: block scores, selection and the cache plan of each unit.
 //
 // NOSA: Native and Offloadable Sparse Attention (paperlayer summary): §3.1
-// (scores from pooled keys; query-aware and query-agnostic selection under a
+// (scores from pooled keys; selection of query-aware and query-agnostic blocks under a
 // minimum overlap), §4 (set difference against the GPU-resident blocks and a
 // replacement mapping).  The arithmetic is that of score_kernel,
 // select_reg_kernel and the planning kernels: the same device functions run

@@ -2,7 +2,7 @@
 
 NOSA: Native and Offloadable Sparse Attention (paperlayer summary, §3.2)
 compares moving selected KV as whole blocks with moving it token by token, at
-batch 64, sequence length 4096, d_kv = 128 and 2 KV heads, as locality rises;
+batch 64 with 4096-token sequences, 128-dim keys and values and two KV heads, as locality rises;
 §4 describes the block transfer as a zero-copy kernel over 16 KiB blocks.
 
 This module measures both with one kernel (``nosa_gather_rows``) on the same

@@ -12,11 +12,11 @@
  *         query-aware and a query-agnostic subset; two-stage block scoring with
  *         mean pooling over sub-blocks then max pooling to the block.
  *  [S21]  same page, §2.1 -- query-aware top-k vs query-agnostic eviction.
- *  [S22]  same page, §2.2 -- locality = fraction of the tokens selected at step t
- *         that were also selected at step t-1.
- *  [S4]   same page, §4 -- set difference between old and new selections gives a
- *         replacement mapping; only blocks unused by the current step are
- *         swapped out; non-contiguous GPU-resident blocks.
+ *  [S22]  same page, §2.2 -- locality: the share of step t's selected tokens
+ *         that step t-1 had selected too.
+ *  [S4]   same page, §4 -- a kernel compares the old and new selections and
+ *         decides which cached blocks give up their slots; blocks the step
+ *         uses keep theirs; cached blocks need not sit contiguously.
  *  [SA]   same page, App. A (pseudocode summary) -- per step: select blocks,
  *         transfer the cache-missed blocks CPU->GPU, attend with the cache.
  *  [SE]   same page, App. E -- |Gamma(t-1) ∩ Gamma(t)| >= k_e.
