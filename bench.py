@@ -593,7 +593,7 @@ MAX_QUERY_STEPS = 16000
 NCU_TRAFFIC = {
     ("gather_attend_kernel", "offload_b64"): {"dram": 592384 + 36096, "pcie_read": 20717568,
                                               "payload": 592348 * 32},
-    ("attend_hits_ws_kernel", "layer8b"): {"dram": 268951808 + 5076480},
+    ("attend_hits_ws_kernel", "layer8b"): {"dram": 268836864 + 3991552},
 }
 
 

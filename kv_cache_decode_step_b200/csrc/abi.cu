@@ -152,6 +152,7 @@ struct nosa_ctx {
   int* own_nfetch = nullptr;
   int attn_stages = 3;      // TMA stages per hits-pass CTA
   bool attn_producer = true;  // hits pass with a producer warp of its own
+  bool kv_evict_first = true; // hits pass K/V loads marked first to leave L2
 };
 
 namespace {
@@ -323,6 +324,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   int want = 2 * sms - (c->offloaded ? c->gather_grid : 0);
   if (want < sms) want = sms;
   if (const char* v = getenv("NOSA_ATTN_PRODUCER")) c->attn_producer = atoi(v) != 0;
+  if (const char* v = getenv("NOSA_KV_EVICT_FIRST")) c->kv_evict_first = atoi(v) != 0;
   if (const char* v = getenv("NOSA_ATTN_STAGES")) c->attn_stages = atoi(v) == 2 ? 2 : 3;
   if (c->attn_stages == 2) want = 3 * sms - (c->offloaded ? c->gather_grid : 0);
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
@@ -761,6 +763,7 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
   a.nparts = c->nparts;
   a.part_base = 0;
   a.hits_grid = c->attn_grid;
+  a.kv_evict_first = c->kv_evict_first ? 1 : 0;
   a.out = static_cast<uint16_t*>(out);
   a.st = c->st;
   a.miss_base = c->hits_parts;

@@ -56,10 +56,18 @@ __device__ __forceinline__ void issue_block(const DecodeMaps& m, const DecodeArg
   unsigned char* kt = sm + st * kStageBytes;
   unsigned char* vt = kt + kBlockBytes;
   mbar_arrive_expect_tx(&bars[st], 2 * kBlockBytes);
-  tma_load_2d(kt, mk, &bars[st], 0, row);
-  tma_load_2d(kt + kHalfBytes, mk, &bars[st], 64, row);
-  tma_load_2d(vt, mv, &bars[st], 0, row);
-  tma_load_2d(vt + kHalfBytes, mv, &bars[st], 64, row);
+  if (a.kv_evict_first) {
+    const uint64_t pol = l2_evict_first_policy();
+    tma_load_2d_hint(kt, mk, &bars[st], 0, row, pol);
+    tma_load_2d_hint(kt + kHalfBytes, mk, &bars[st], 64, row, pol);
+    tma_load_2d_hint(vt, mv, &bars[st], 0, row, pol);
+    tma_load_2d_hint(vt + kHalfBytes, mv, &bars[st], 64, row, pol);
+  } else {
+    tma_load_2d(kt, mk, &bars[st], 0, row);
+    tma_load_2d(kt + kHalfBytes, mk, &bars[st], 64, row);
+    tma_load_2d(vt, mv, &bars[st], 0, row);
+    tma_load_2d(vt + kHalfBytes, mv, &bars[st], 64, row);
+  }
 }
 
 __device__ __forceinline__ bool position_valid(const DecodeArgs& a, int j, int n_hit_u, int tail_len) {

@@ -106,6 +106,25 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// The same load with an L2 cache policy (see l2_evict_first_policy).
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// An L2 policy that makes the lines a load brings in the first to go: for
+// data read once per step (the selected K/V), so that data reused across
+// steps (the pooled keys) stays in L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // Untiled bulk copy global -> shared (no multicast), completing on an
 // mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -325,6 +344,7 @@ struct DecodeArgs {
   int part_base, nparts;    // hits pass writes slots part_base + segment; nparts per unit
   int miss_base;            // slot of a unit's first fetched-block partial
   int hits_grid;            // CTAs of the hits pass (fixes each unit's segment count)
+  int kv_evict_first;       // 1: the hits pass loads K/V with the L2 evict-first policy
   int* unit_done;           // [U] partials written this step; completing one merges the unit
   uint16_t* out;            // [B, Hq, d]
   int* done_ctr;            // non-null: units merged; the last merge ends the step (advance_step)
