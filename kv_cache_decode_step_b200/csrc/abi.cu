@@ -153,6 +153,7 @@ struct nosa_ctx {
   int attn_stages = 3;      // TMA stages per hits-pass CTA
   bool attn_producer = true;  // hits pass with a producer warp of its own
   bool kv_evict_first = true; // hits pass K/V loads marked first to leave L2
+  bool pdl = true;            // gather placed while the plan finishes (programmatic dependent launch)
 };
 
 namespace {
@@ -325,6 +326,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   if (want < sms) want = sms;
   if (const char* v = getenv("NOSA_ATTN_PRODUCER")) c->attn_producer = atoi(v) != 0;
   if (const char* v = getenv("NOSA_KV_EVICT_FIRST")) c->kv_evict_first = atoi(v) != 0;
+  if (const char* v = getenv("NOSA_PDL")) c->pdl = atoi(v) != 0;
   if (const char* v = getenv("NOSA_ATTN_STAGES")) c->attn_stages = atoi(v) == 2 ? 2 : 3;
   if (c->attn_stages == 2) want = 3 * sms - (c->offloaded ? c->gather_grid : 0);
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
@@ -689,7 +691,7 @@ nosa_status nosa_score_select_fetch(nosa_ctx* c, const void* q, double* scores, 
       return s;
     }
     NOSA_CUDA(launch_select_plan(select_args(c, scores, sel), plan_args(c, sel, fetch, n_fetch), c->offloaded ? 1 : 0,
-                                 reinterpret_cast<cudaStream_t>(compute)));
+                                 reinterpret_cast<cudaStream_t>(compute), c->pdl));
     c->copy_stream = reinterpret_cast<cudaStream_t>(copy);
     c->gather_on_side = c->offloaded && copy != compute;
     c->phase = kFetched;
@@ -795,13 +797,13 @@ nosa_status nosa_sparse_decode(nosa_ctx* c, const void* q, const int32_t* sel, v
       // the gather goes first, on this stream, so its CTAs are placed before
       // the hits pass's; the hits pass runs beside it on the second stream
       NOSA_CUDA(cudaEventRecord(c->ev_plan, st));
-      NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, st));
+      NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, st, c->pdl));
       NOSA_CUDA(cudaStreamWaitEvent(c->copy_stream, c->ev_plan, 0));
       NOSA_CUDA(launch_attend_hits(a, c->maps, c->attn_grid, c->copy_stream, c->attn_stages, c->attn_producer));
       NOSA_CUDA(cudaEventRecord(c->ev_gather, c->copy_stream));
       NOSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
     } else {
-      NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, st));
+      NOSA_CUDA(launch_gather_attend(ga, c->gather_grid, st, c->pdl));
     }
   }
   // hits pass: blocks already on the GPU (all of S(t) when KV is in HBM) plus

@@ -21,7 +21,10 @@
 // larger copy role.
 // The roles hand stages over with named barriers (FULL: copy -> attention,
 // EMPTY: attention -> copy), the entry riding with the stage, so every
-// barrier phase has all its arrivals.  Nothing waits on another CTA or kernel.
+// barrier phase has all its arrivals.  Nothing waits on another CTA.  The
+// kernel may be launched as a programmatic dependent of the planning kernel:
+// its CTAs are then placed while the plan finishes and read the plan only
+// after it has completed.
 #include "attend_dev.cuh"
 
 namespace nosa {
@@ -61,6 +64,7 @@ __global__ void __launch_bounds__(kGaThreads, 1) gather_attend_kernel(GatherAtte
   const int warp = rt >> 5, lane = threadIdx.x & 31;
   const WarpStates ws(ga_smem + kGaStages * kGaStageBytes);
   int* flag = reinterpret_cast<int*>(ga_smem + kGaStages * kGaStageBytes + kGaWsBytes);
+  grid_dep_wait();  // the plan (list, count, counters) is complete and visible
   // one read of the list length and of the staged block for the whole CTA
   // (the last unit merged of the step clears the count)
   int* s_entry = flag + 4;  // entry claimed for stage 0, 1
@@ -160,21 +164,11 @@ cudaError_t configure_gather_attend() {
 
 // Launched with the device's highest CTA priority so that its few CTAs are
 // dispatched ahead of the hits pass running beside it.
-cudaError_t launch_gather_attend(const GatherAttendArgs& a, int grid, cudaStream_t st) {
+cudaError_t launch_gather_attend(const GatherAttendArgs& a, int grid, cudaStream_t st, bool pdl) {
   int least = 0, greatest = 0;
   cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kGaThreads);
-  cfg.dynamicSmemBytes = kGaSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributePriority;
-  attr[0].val.priority = greatest;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gather_attend_kernel, a);
+  return launch_ex(gather_attend_kernel, dim3(grid), dim3(kGaThreads), kGaSmemBytes, st, pdl, greatest, a);
 }
 
 }  // namespace nosa

@@ -58,6 +58,17 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may have its CTAs placed while the kernel
+// before it on the stream is still running; grid_dep_wait() returns once that
+// kernel has completed and its writes are visible, so everything a kernel
+// reads from its predecessor comes after it.  Launched without the attribute,
+// the wait returns at once.  grid_dep_launch() lets such a dependent be placed
+// as soon as every CTA of this grid has issued it (or exited); the dependent's
+// CTAs then wait on the SMs instead of being launched after the completion.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
@@ -311,8 +322,11 @@ bool prepare_supported(int max_blocks);
 cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t st);
 // Selection and plan in one launch (one warp per unit), after score_kernel;
 // for max_blocks <= 1024.  Same results as launch_select then launch_plan.
+// pdl: launched as a programmatic dependent of the kernel before it on `st`
+// (the score kernel, which lets its dependents be placed early).
 bool select_plan_supported(int max_blocks);
-cudaError_t launch_select_plan(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st);
+cudaError_t launch_select_plan(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st,
+                               bool pdl = false);
 
 struct GatherArgs {
   const uint16_t* hk;       // host K (device-addressable), [U, max_blocks*P, d]
@@ -377,7 +391,35 @@ struct GatherAttendArgs {
   GatherArgs g;
   DecodeArgs d;
 };
-cudaError_t launch_gather_attend(const GatherAttendArgs& a, int grid, cudaStream_t st);
+cudaError_t launch_gather_attend(const GatherAttendArgs& a, int grid, cudaStream_t st, bool pdl = false);
+
+// Launch of `kernel` on `st`; with pdl, as a programmatic dependent of the
+// kernel before it on the stream (the kernel must call grid_dep_wait() before
+// it reads anything that kernel writes); priority: CTA priority, or 0.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                      int priority, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (priority != 0) {
+    attr[n].id = cudaLaunchAttributePriority;
+    attr[n].val.priority = priority;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
 
 // Named barriers (bar.sync / bar.arrive over `count` threads, whole warps).
 __device__ __forceinline__ void bar_sync(int id, int count) {

@@ -41,6 +41,9 @@ __global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs
   int* s_bs = s_lu + 32;  // general plan: the unit's block -> slot table [max_blocks]
   const int u = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the gather that follows may be placed now: it waits for this kernel's
+  // completion before it reads anything
+  grid_dep_launch();
   // the gather that follows claims its entries from 0 (it is the only user
   // of this counter and runs after this kernel has completed)
   if (u == 0 && threadIdx.x == 0) a.sc.ds->gather_next = 0;
@@ -119,6 +122,8 @@ __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectA
   __shared__ int ssrc[kSelPlanWarps][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * kSelPlanWarps + warp;
+  grid_dep_wait();    // the scores are complete
+  grid_dep_launch();  // the gather that follows may be placed
   // the gather that follows claims its entries from 0
   if (blockIdx.x == 0 && threadIdx.x == 0) se.ds->gather_next = 0;
   if (u >= se.U) return;
@@ -152,7 +157,8 @@ __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectA
 }
 
 template <int R>
-cudaError_t launch_select_plan_r(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st) {
+cudaError_t launch_select_plan_r(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st,
+                                 bool pdl) {
   const bool reg_plan = offloaded && pl.C <= 32 && pl.k <= 32;
   const int wide_ints = se.k + (!offloaded ? 0 : reg_plan ? 64 : 2 * pl.C + 2 * pl.k + pl.max_blocks);
   const size_t smem = (size_t)kSelPlanWarps * wide_ints * sizeof(int);
@@ -162,16 +168,17 @@ cudaError_t launch_select_plan_r(const SelectArgs& se, const PlanArgs& pl, int o
     if (e != cudaSuccess) return e;
   }
   const int grid = (se.U + kSelPlanWarps - 1) / kSelPlanWarps;
-  select_plan_kernel<R><<<grid, kSelPlanWarps * 32, smem, st>>>(se, pl, offloaded, wide_ints);
-  return cudaGetLastError();
+  return launch_ex(select_plan_kernel<R>, dim3(grid), dim3(kSelPlanWarps * 32), smem, st, pdl, 0, se, pl, offloaded,
+                   wide_ints);
 }
 
 bool select_plan_supported(int max_blocks) { return max_blocks <= 1024; }
 
-cudaError_t launch_select_plan(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st) {
+cudaError_t launch_select_plan(const SelectArgs& se, const PlanArgs& pl, int offloaded, cudaStream_t st,
+                               bool pdl) {
   const int rows = (se.max_blocks + 31) / 32;
-  if (rows <= 16) return launch_select_plan_r<16>(se, pl, offloaded, st);
-  if (rows <= 32) return launch_select_plan_r<32>(se, pl, offloaded, st);
+  if (rows <= 16) return launch_select_plan_r<16>(se, pl, offloaded, st, pdl);
+  if (rows <= 32) return launch_select_plan_r<32>(se, pl, offloaded, st, pdl);
   return cudaErrorInvalidValue;
 }
 

@@ -72,6 +72,7 @@ constexpr uint64_t kScoreWaitNs = 1000000000ull;
 __global__ void __launch_bounds__(kScoreWarps * 32) score_kernel(ScoreArgs a) {
   __shared__ __align__(128) uint4 skb[kScoreCtaBlocks * kBlockU4];  // 32 KiB
   __shared__ __align__(8) uint64_t bars[kScoreWarps];
+  grid_dep_launch();  // a selection launched as a dependent may be placed; it waits for the scores
   const int u = blockIdx.y;
   const int n = a.ds->n_closed;
   const int j0 = blockIdx.x * kScoreCtaBlocks;
