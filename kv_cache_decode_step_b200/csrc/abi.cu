@@ -154,6 +154,7 @@ struct nosa_ctx {
   bool attn_producer = true;  // hits pass with a producer warp of its own
   bool kv_evict_first = true; // hits pass K/V loads marked first to leave L2
   bool pdl = true;            // gather placed while the plan finishes (programmatic dependent launch)
+  bool placed_widen = true;   // scoring widens half of the pooled keys by bit placement
 };
 
 namespace {
@@ -327,6 +328,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   if (const char* v = getenv("NOSA_ATTN_PRODUCER")) c->attn_producer = atoi(v) != 0;
   if (const char* v = getenv("NOSA_KV_EVICT_FIRST")) c->kv_evict_first = atoi(v) != 0;
   if (const char* v = getenv("NOSA_PDL")) c->pdl = atoi(v) != 0;
+  if (const char* v = getenv("NOSA_PLACED_WIDEN")) c->placed_widen = atoi(v) != 0;
   if (const char* v = getenv("NOSA_ATTN_STAGES")) c->attn_stages = atoi(v) == 2 ? 2 : 3;
   if (c->attn_stages == 2) want = 3 * sms - (c->offloaded ? c->gather_grid : 0);
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
@@ -537,6 +539,7 @@ ScoreArgs score_args(const nosa_ctx* c, const void* q, double* scores) {
   a.Hkv = c->cfg.n_kv_heads;
   a.G = c->G;
   a.max_blocks = c->max_blocks;
+  a.placed_widen = c->placed_widen ? 1 : 0;
   return a;
 }
 

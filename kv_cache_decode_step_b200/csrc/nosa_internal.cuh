@@ -212,6 +212,20 @@ __device__ __forceinline__ double bf16_lo_to_f64(uint32_t w) { return (double)__
 __device__ __forceinline__ double bf16_hi_to_f64(uint32_t w) {
   return (double)__uint_as_float(w & 0xFFFF0000u);
 }
+// The upper bf16 of w times 2^-896, exactly, without a conversion
+// instruction: its sign, 8 exponent bits and 7 fraction bits placed in the
+// fp64 high word so that the 8-bit exponent sits in the low bits of the
+// 11-bit field (3 bits lower than bf16 -> fp32 places it).  The fp64 bias
+// (1023) exceeds bf16's (127) by 896, so a normal bf16 keeps its fraction and
+// loses 2^896 of scale, and a zero or subnormal bf16 (exponent 0) becomes the
+// fp64 zero or subnormal of the same fraction, again 2^896 smaller.  A product
+// with an operand scaled up by 2^896 is therefore the same real number as the
+// unscaled product and rounds identically.  Finite inputs only.
+constexpr double kBf16PlaceScale = 0x1p896;
+__device__ __forceinline__ double bf16_hi_placed_f64(uint32_t w) {
+  const uint32_t hi = ((w & 0x7FFF0000u) >> 3) | (w & 0x80000000u);
+  return __hiloint2double((int)hi, 0);
+}
 
 // fp64 -> bf16 with round-to-nearest-even, by integer rounding of the fp64
 // significand to the bf16 grid (8 significant bits; spacing 2^-133 below
@@ -273,6 +287,7 @@ struct ScoreArgs {
   double* scores;           // [U, max_blocks]
   DevState* ds;
   int U, Hq, Hkv, G, max_blocks;
+  int placed_widen;         // 1: half of the keys widened by bit placement (same results)
 };
 cudaError_t launch_score(const ScoreArgs& a, cudaStream_t st);
 

@@ -107,24 +107,25 @@ __global__ void __launch_bounds__(kScoreWarps * 32) score_kernel(ScoreArgs a) {
       timed_out = true;
     } else {
       double sres[kScoreWarpBlocks];
+      auto dots = [&](auto placed) {
+        constexpr bool kPlaced = decltype(placed)::value;
 #pragma unroll
-      for (int i = 0; i < kScoreWarpBlocks; ++i) {
-        if (i < cnt) {
-          const uint4* row = skb + (jw + i) * kBlockU4 + r * kRowU4;
-          sres[i] = dot16(row[c], row[8 + c], qt);
-        } else {
-          sres[i] = 0.0;
+        for (int i = 0; i < kScoreWarpBlocks; ++i) {
+          if (i < cnt) {
+            const uint4* row = skb + (jw + i) * kBlockU4 + r * kRowU4;
+            sres[i] = dot16<kPlaced>(row[c], row[8 + c], qt);
+          } else {
+            sres[i] = 0.0;
+          }
         }
+      };
+      if (a.placed_widen && place_query_terms(qt)) {
+        dots(std::true_type{});
+      } else {
+        dots(std::false_type{});
       }
-#pragma unroll
-      for (int i = 0; i < kScoreWarpBlocks; ++i) sres[i] = block_reduce(sres[i]);
-      if (lane < cnt) {
-        double v = sres[0];
-#pragma unroll
-        for (int i = 1; i < kScoreWarpBlocks; ++i)
-          if (lane == i) v = sres[i];
-        a.scores[(size_t)u * a.max_blocks + j0 + jw + lane] = v;
-      }
+      const double v = blocks_reduce<kScoreWarpBlocks>(sres, lane);
+      if (lane < cnt) a.scores[(size_t)u * a.max_blocks + j0 + jw + lane] = v;
     }
   }
   // never leave a bulk copy in flight behind an exiting CTA

@@ -10,33 +10,87 @@
 // whose products are exact.
 #pragma once
 
+#include <type_traits>
+
 #include "nosa_internal.cuh"
 
 namespace nosa {
 
 constexpr int kBlockU4 = kR * kRowU4;  // 16-byte words of pooled keys per block (64)
 
-__device__ __forceinline__ double dot16(const uint4& a, const uint4& b, const double* qt) {
-  double s = 0.0;
-  s = fma(qt[0], bf16_lo_to_f64(a.x), s);  s = fma(qt[1], bf16_hi_to_f64(a.x), s);
-  s = fma(qt[2], bf16_lo_to_f64(a.y), s);  s = fma(qt[3], bf16_hi_to_f64(a.y), s);
-  s = fma(qt[4], bf16_lo_to_f64(a.z), s);  s = fma(qt[5], bf16_hi_to_f64(a.z), s);
-  s = fma(qt[6], bf16_lo_to_f64(a.w), s);  s = fma(qt[7], bf16_hi_to_f64(a.w), s);
-  s = fma(qt[8], bf16_lo_to_f64(b.x), s);  s = fma(qt[9], bf16_hi_to_f64(b.x), s);
-  s = fma(qt[10], bf16_lo_to_f64(b.y), s); s = fma(qt[11], bf16_hi_to_f64(b.y), s);
-  s = fma(qt[12], bf16_lo_to_f64(b.z), s); s = fma(qt[13], bf16_hi_to_f64(b.z), s);
-  s = fma(qt[14], bf16_lo_to_f64(b.w), s); s = fma(qt[15], bf16_hi_to_f64(b.w), s);
+// One 16-byte word's contribution (dims 2i .. 2i+7 of qt), fma by fma.  With
+// kPlaced the upper bf16 of each 32-bit word is widened by bit placement
+// (bf16_hi_placed_f64) and its query term qt[2i+1] is expected scaled by
+// 2^896: the fp64 pipe, which also runs the conversions, then widens only
+// half of the keys, the other half goes to the integer pipe, and every fma
+// rounds exactly as with two conversions.
+template <bool kPlaced>
+__device__ __forceinline__ double dot8_acc(const uint4& a, const double* qt, double s) {
+  const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    s = fma(qt[2 * i], bf16_lo_to_f64(wv[i]), s);
+    s = fma(qt[2 * i + 1], kPlaced ? bf16_hi_placed_f64(wv[i]) : bf16_hi_to_f64(wv[i]), s);
+  }
   return s;
 }
 
-__device__ __forceinline__ double block_reduce(double s) {
-  s += __shfl_xor_sync(0xffffffffu, s, 1);
-  s += __shfl_xor_sync(0xffffffffu, s, 2);
-  s += __shfl_xor_sync(0xffffffffu, s, 4);
-  double o = __shfl_xor_sync(0xffffffffu, s, 8);
-  s = o > s ? o : s;
-  o = __shfl_xor_sync(0xffffffffu, s, 16);
-  return o > s ? o : s;
+template <bool kPlaced>
+__device__ __forceinline__ double dot16(const uint4& a, const uint4& b, const double* qt) {
+  return dot8_acc<kPlaced>(b, qt + 8, dot8_acc<kPlaced>(a, qt, 0.0));
+}
+
+// Whether this warp may use placed widening: every lane's odd query sums,
+// scaled by 2^896, stay finite (|qt| < 2^126 leaves a margin).  If so, they
+// are scaled in place.  Warp-wide vote: both paths give the same bits.
+__device__ __forceinline__ bool place_query_terms(double (&qt)[16]) {
+  bool ok = true;
+#pragma unroll
+  for (int i = 1; i < 16; i += 2) ok = ok && fabs(qt[i]) < 0x1p126;
+  ok = __all_sync(0xffffffffu, ok);
+  if (ok) {
+#pragma unroll
+    for (int i = 1; i < 16; i += 2) qt[i] *= kBf16PlaceScale;
+  }
+  return ok;
+}
+
+// Scores of NB blocks (NB = 4 or 8) from this lane's partial sums s[i] of
+// block i: the sum over the 8 lanes of each sub-block, then the max over the
+// 4 sub-blocks.  The sums halve the values per lane at each step: across
+// lanes l and l ^ d a lane keeps the blocks whose index bit matches its own
+// lane bit and sends the others to its partner, so after the steps d = 1, 2, 4
+// lane 8r + c holds sub-block r's sum of block c % NB.  Every sum pairs the
+// same operands as a butterfly over each block in turn, so the results are
+// the same bits.  Lanes c % NB = i return block i's score.
+template <int NB>
+__device__ __forceinline__ double blocks_reduce(const double (&s)[NB], int lane) {
+  static_assert(NB == 4 || NB == 8, "4 or 8 blocks");
+  double v[NB];
+#pragma unroll
+  for (int i = 0; i < NB; ++i) v[i] = s[i];
+  int m = NB;
+#pragma unroll
+  for (int d = 1; d < 8; d <<= 1) {
+    if (m > 1) {
+      const bool odd = (lane & d) != 0;
+#pragma unroll
+      for (int i = 0; i < NB / 2; ++i) {
+        if (i < m / 2) {
+          const double keep = odd ? v[2 * i + 1] : v[2 * i];
+          const double send = odd ? v[2 * i] : v[2 * i + 1];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+        }
+      }
+      m /= 2;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], d);
+    }
+  }
+  double o = __shfl_xor_sync(0xffffffffu, v[0], 8);
+  double x = o > v[0] ? o : v[0];
+  o = __shfl_xor_sync(0xffffffffu, x, 16);
+  return o > x ? o : x;
 }
 
 // qt = sum over the unit's G query heads of their dims [8c, 8c+8) and
@@ -73,19 +127,15 @@ __device__ __forceinline__ void score_group_load(const uint4* base, int g0, int 
   }
 }
 
+template <bool kPlaced>
 __device__ __forceinline__ void score_group_finish(const ScoreArgs& a, int u, int g0, int cnt, int lane,
                                                    const uint4 (&x)[4], const uint4 (&y)[4], const double (&qt)[16],
                                                    double* sc_out) {
   double sres[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) sres[i] = i < cnt ? dot16(x[i], y[i], qt) : 0.0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) sres[i] = block_reduce(sres[i]);
+  for (int i = 0; i < 4; ++i) sres[i] = i < cnt ? dot16<kPlaced>(x[i], y[i], qt) : 0.0;
+  const double v = blocks_reduce<4>(sres, lane);
   if (lane < cnt) {
-    double v = sres[0];
-#pragma unroll
-    for (int i = 1; i < 4; ++i)
-      if (lane == i) v = sres[i];
     sc_out[g0 + lane] = v;
     a.scores[(size_t)u * a.max_blocks + g0 + lane] = v;
   }
@@ -128,16 +178,24 @@ __device__ __forceinline__ void score_unit_warps(const ScoreArgs& a, int u, int 
     group_query_sum(a, u / a.Hkv, u % a.Hkv, c, qt);
   }
   // two groups in flight: each finished group's buffer takes the group after next
-  while (g < n) {
-    score_group_finish(a, u, g, min(4, n - g), lane, xa, ya, qt, sc_out);
-    const int g2 = g1 + stride;
-    if (g2 < n) score_group_load(base, g2, min(4, n - g2), c, xa, ya);
-    if (g1 >= n) break;
-    score_group_finish(a, u, g1, min(4, n - g1), lane, xb, yb, qt, sc_out);
-    const int g3 = g2 + stride;
-    if (g3 < n) score_group_load(base, g3, min(4, n - g3), c, xb, yb);
-    g = g2;
-    g1 = g3;
+  auto groups = [&](auto placed) {
+    constexpr bool kPlaced = decltype(placed)::value;
+    while (g < n) {
+      score_group_finish<kPlaced>(a, u, g, min(4, n - g), lane, xa, ya, qt, sc_out);
+      const int g2 = g1 + stride;
+      if (g2 < n) score_group_load(base, g2, min(4, n - g2), c, xa, ya);
+      if (g1 >= n) break;
+      score_group_finish<kPlaced>(a, u, g1, min(4, n - g1), lane, xb, yb, qt, sc_out);
+      const int g3 = g2 + stride;
+      if (g3 < n) score_group_load(base, g3, min(4, n - g3), c, xb, yb);
+      g = g2;
+      g1 = g3;
+    }
+  };
+  if (a.placed_widen && place_query_terms(qt)) {
+    groups(std::true_type{});
+  } else {
+    groups(std::false_type{});
   }
 }
 

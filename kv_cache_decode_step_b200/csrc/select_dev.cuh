@@ -46,9 +46,22 @@ __device__ __forceinline__ void keep_best_reg(uint32_t& mask, int c, const unsig
   if (left <= c) return;
   uint32_t kept = 0u, cand = mask;
   int need = c;
+  // Key bits on which all members agree split nothing (every member goes the
+  // same way): the search starts at the highest bit where two members differ.
+  unsigned long long k_and = ~0ull, k_or = 0ull;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    if ((mask >> i) & 1u) {
+      k_and &= k[i];
+      k_or |= k[i];
+    }
+  }
+  const unsigned d_hi = __reduce_or_sync(kFull, (unsigned)(k_or >> 32)) & ~__reduce_and_sync(kFull, (unsigned)(k_and >> 32));
+  const unsigned d_lo = __reduce_or_sync(kFull, (unsigned)k_or) & ~__reduce_and_sync(kFull, (unsigned)k_and);
+  const int b_top = d_hi ? 63 - __clz(d_hi) : (d_lo ? 31 - __clz(d_lo) : -1);
   // 64 key bits: the high words, then the low words
 #pragma unroll 1
-  for (int b = 63; b >= 0 && need > 0 && need < left; --b) {
+  for (int b = b_top; b >= 0 && need > 0 && need < left; --b) {
     uint32_t ones = 0u;
 #pragma unroll
     for (int i = 0; i < R; ++i) ones |= (uint32_t)((k[i] >> b) & 1ull) << i;

@@ -37,8 +37,7 @@ def _workload_and_data(n_units_needed):
     return w, data
 
 
-@pytest.mark.parametrize("fused", [True, False])
-def test_scores_cover_every_finite_bf16_pattern(fused):
+def _pattern_case():
     pats = _finite_patterns()                                   # 65,280 patterns
     blocks_needed = -(-len(pats) // 128)
     w, data = _workload_and_data(-(-blocks_needed // 64))
@@ -52,14 +51,27 @@ def test_scores_cover_every_finite_bf16_pattern(fused):
     k[:, : n * 64] = blk.reshape(U, n * 64, d)
     data["k"] = k
     data["q"][:] = 0x3F80                                       # every query 1.0
+    return w, data, rows
+
+
+def _step_scores(w, data, fused):
     dec = runner.Decoder(w, data, fused=fused)
     try:
         dec.step()
         dec.stream.synchronize()
-        got = dec.scores.cpu().numpy()[:, :n]
+        got = dec.scores.cpu().numpy()[:, : w.n_blocks0]
         dec.check()
     finally:
         dec.close()
+    return got
+
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_scores_cover_every_finite_bf16_pattern(fused):
+    w, data, rows = _pattern_case()
+    U, d, n = w.units, w.head_dim, w.n_blocks0
+    k = data["k"]
+    got = _step_scores(w, data, fused)
     q1 = np.full((w.group, d), 0x3F80, dtype=np.uint16)
     for u in range(U):
         kbar = oracle.pool_keys(k[u, : n * 64], 16)
@@ -68,3 +80,44 @@ def test_scores_cover_every_finite_bf16_pattern(fused):
         bound = 4 * np.abs(vals).sum(axis=1) * 128 * 2.0 ** -52
         assert np.all(np.abs(got[u] - want) <= bound), u
         assert np.array_equal(got[u] == 0.0, want == 0.0)
+
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_placed_widening_gives_the_bits_of_conversions(fused, monkeypatch):
+    """Half of the keys are widened by placing their bits in the fp64 high
+    word (a value 2^896 smaller, the query term 2^896 larger): over every
+    finite bf16 pattern the scores are bit-identical to widening every key
+    by conversion (NOSA_PLACED_WIDEN=0)."""
+    w, data, _ = _pattern_case()
+    got = _step_scores(w, data, fused)
+    monkeypatch.setenv("NOSA_PLACED_WIDEN", "0")
+    want = _step_scores(w, data, fused)
+    assert np.array_equal(got.view(np.uint64), want.view(np.uint64))
+
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_queries_too_large_for_placement(fused, monkeypatch):
+    """Group sums of 2^126 or more would overflow once scaled by 2^896: those
+    warps widen by conversion, and the scores still match the oracle and the
+    conversion-only path bit for bit."""
+    w = configs.get("tiny", batch=2, offloaded=False, cache_factor=0, steps=2)
+    data = inputs.generate(w)
+    q = data["q"]                             # [units, steps, group, d]
+    q[0, 0] = 0x7E80                          # 8.5e37 in every head of unit 0 at step 0: the group sum > 2^126
+    q[0, 0, :, 1::7] = 0xFE80                 # some of them negative
+    got = _step_scores(w, data, fused)
+    monkeypatch.setenv("NOSA_PLACED_WIDEN", "0")
+    want = _step_scores(w, data, fused)
+    assert np.array_equal(got.view(np.uint64), want.view(np.uint64))
+
+    def widen(bits):
+        return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    n = w.n_blocks0
+    for u in range(w.units):
+        kbar = oracle.pool_keys(data["k"][u, : n * 64], 16)
+        ref = oracle.score_blocks(q[u, 0], kbar, 4)
+        # fp64 rounding of 128-term sums of exact products
+        qt = widen(q[u, 0]).sum(axis=0)
+        terms = np.abs(widen(kbar).reshape(n, 4, -1) * qt).sum(axis=2).max(axis=1)
+        assert np.all(np.abs(got[u] - ref) <= terms * 128 * 2.0 ** -52), u
