@@ -155,6 +155,7 @@ struct nosa_ctx {
   bool kv_evict_first = true; // hits pass K/V loads marked first to leave L2
   bool pdl = true;            // gather placed while the plan finishes (programmatic dependent launch)
   bool placed_widen = true;   // scoring widens half of the pooled keys by bit placement
+  int warm_blocks = 12;       // KV in HBM: blocks per hits-pass CTA asked of L2 during the selection
 };
 
 namespace {
@@ -329,6 +330,7 @@ nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out) {
   if (const char* v = getenv("NOSA_KV_EVICT_FIRST")) c->kv_evict_first = atoi(v) != 0;
   if (const char* v = getenv("NOSA_PDL")) c->pdl = atoi(v) != 0;
   if (const char* v = getenv("NOSA_PLACED_WIDEN")) c->placed_widen = atoi(v) != 0;
+  if (const char* v = getenv("NOSA_WARM_BLOCKS")) c->warm_blocks = atoi(v) < 0 ? 0 : (atoi(v) > 64 ? 64 : atoi(v));
   if (const char* v = getenv("NOSA_ATTN_STAGES")) c->attn_stages = atoi(v) == 2 ? 2 : 3;
   if (c->attn_stages == 2) want = 3 * sms - (c->offloaded ? c->gather_grid : 0);
   if (const char* v = getenv("NOSA_ATTN_CTAS")) want = atoi(v) > 0 ? atoi(v) : want;
@@ -666,6 +668,13 @@ nosa_status fused_first_half(nosa_ctx* c, const void* q, uint16_t* q_copy, doubl
   a.pl = plan_args(c, sel, fetch, n_fetch);
   a.offloaded = c->offloaded ? 1 : 0;
   a.nwarps = c->prep_warps;
+  if (!c->offloaded && c->warm_blocks > 0) {
+    a.warm_k = c->kv_k;
+    a.warm_v = c->kv_v;
+    a.warm_blocks = c->warm_blocks;
+    a.hits_vpu = c->hits_vpu;
+    a.hits_grid = c->attn_grid;
+  }
   NOSA_CUDA(launch_prepare(a, cs));
   c->copy_stream = xs;
   c->gather_on_side = c->offloaded && xs != cs;

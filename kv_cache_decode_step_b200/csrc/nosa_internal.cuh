@@ -136,6 +136,13 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return p;
 }
 
+// Bulk prefetch of global memory into L2 (no data reaches the SM).  Address
+// 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
+
 // Untiled bulk copy global -> shared (no multicast), completing on an
 // mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -332,6 +339,12 @@ struct PrepareArgs {
   int offloaded;
   int nwarps;               // warps per CTA (4..16): more when there are few units
   int plan_ints;            // set by the launcher
+  // KV in HBM: while warp 0 selects, warp 1 asks L2 for the blocks that the
+  // hits-pass CTAs starting in this unit load first (warm_blocks each), as
+  // S(t-1) places them (S(t) keeps at least m of its blocks).  Null: off.
+  const uint16_t* warm_k;   // resident K / V [U, max_blocks*P, d]
+  const uint16_t* warm_v;
+  int warm_blocks, hits_vpu, hits_grid;
 };
 bool prepare_supported(int max_blocks);
 cudaError_t launch_prepare(const PrepareArgs& a, cudaStream_t st);

@@ -25,6 +25,34 @@ constexpr int kPrepMaxThreads = 512;
 // [32] x 2 and the general plan's block -> slot table [max_blocks].  The
 // copies are loaded while the scores stream in, so selection and planning
 // read no global memory of their own.
+// Warp-wide: L2 prefetches of the first warm_blocks positions of every
+// hits-pass CTA whose range starts in unit u, with the block ids of S(t-1)
+// (prev: the unit's copy in shared memory).  The hits pass walks positions
+// u * vpu + j (j < k: the j-th selected block) and CTA c starts at
+// floor(c * U * vpu / grid).  A hint only: nothing reads what it brings in
+// unless the pass loads the same block.
+__device__ __forceinline__ void warm_first_blocks(const PrepareArgs& a, int u, int lane, const int* prev) {
+  if (a.sc.ds->step == 0) return;  // no S(t-1) yet
+  const long long V = (long long)a.sc.U * a.hits_vpu;
+  const long long p0 = (long long)u * a.hits_vpu, p1 = p0 + a.hits_vpu;
+  const int c0 = (int)((p0 * a.hits_grid + V - 1) / V);  // first CTA with start >= p0
+  for (int i = lane;; i += 32) {
+    const int c = c0 + i / a.warm_blocks;
+    if (c >= a.hits_grid) break;
+    const long long s = (long long)c * V / a.hits_grid;
+    if (s >= p1) break;
+    const long long p = s + i % a.warm_blocks;
+    if (p >= (long long)(c + 1) * V / a.hits_grid) continue;
+    const int j = (int)(p - p0);
+    if (j >= a.se.k) continue;
+    const int blk = prev[j];
+    if (blk < 0 || blk >= a.sc.max_blocks) continue;
+    const size_t off = ((size_t)u * a.sc.max_blocks + blk) * kP * kD;
+    bulk_prefetch_l2(a.warm_k + off, kBlockBytes);
+    bulk_prefetch_l2(a.warm_v + off, kBlockBytes);
+  }
+}
+
 template <int R>
 __global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs a) {
   extern __shared__ __align__(16) unsigned char prep_smem[];
@@ -70,7 +98,10 @@ __global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs
   score_unit_warps(a.sc, u, warp, blockDim.x >> 5, lane, ssc, s_q);
   cp_async_wait_all();
   __syncthreads();
-  if (warp != 0) return;
+  if (warp != 0) {
+    if (warp == 1 && a.warm_k) warm_first_blocks(a, u, lane, s_prev);
+    return;
+  }
 
   select_unit_reg<R>(a.se, u, lane, sbm, ssc, s_prev, s_ge, s_sel);
   __syncwarp();  // the selection is read back by the plan
