@@ -587,13 +587,16 @@ APPEND_TIMED_STEPS = 2400  # most timed steps of a growing workload (its KV capa
 QUERY_BUDGET_BYTES = 3.5e9  # queries of an offloaded run (on the device, and pinned for the end-to-end pass)
 MAX_QUERY_STEPS = 16000
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu --set
-# full capture of the dominant kernel on its workload (pcie: link-level read
-# bytes, the traffic that bounds the gather).  Retake after changing the kernel.
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one single-pass
+# ncu capture of the dominant kernel on its workload (pcie: link-level read
+# bytes, the traffic that bounds the gather; payload: the host-memory sectors
+# the same launch read).  The hits pass was captured with the caches left as the
+# step leaves them (--cache-control none), so its DRAM bytes are those read
+# inside its own launch.  Retake after changing the kernel.
 NCU_TRAFFIC = {
-    ("gather_attend_kernel", "offload_b64"): {"dram": 592384 + 36096, "pcie_read": 20717568,
-                                              "payload": 592348 * 32},
-    ("attend_hits_ws_kernel", "layer8b"): {"dram": 268836864 + 3991552},
+    ("gather_attend_kernel", "offload_b64"): {"dram": 591616 + 31744, "pcie_read": 20726784,
+                                              "payload": 593076 * 32},
+    ("attend_hits_ws_kernel", "layer8b"): {"dram": 261179904 + 0},
 }
 
 
