@@ -140,15 +140,17 @@ bool prepare_supported(int max_blocks) { return max_blocks <= kPrepareMaxBlocks;
 // selection in shared memory.  The unit's slot tables (and, for the general
 // plan, its block -> slot table) arrive in shared memory by cp.async while
 // the selection runs, so the plan reads no global memory of its own.
-// Shared memory per warp (wide_ints): the selection [k], then the general
-// plan's scratch (2C + 2k ints, slot tables first) and block -> slot table
-// [max_blocks], or the register plan's slot tables [32] x 2.
+// Shared memory: each warp's copy of its unit's scores [sc_stride] fp64 (read
+// from global memory in one burst of 16-byte copies rather than one load per
+// block and lane), then per warp (wide_ints): the selection [k], then the
+// general plan's scratch (2C + 2k ints, slot tables first) and block -> slot
+// table [max_blocks], or the register plan's slot tables [32] x 2.
 constexpr int kSelPlanWarps = 4;
 
 template <int R>
 __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectArgs se, PlanArgs pl, int offloaded,
-                                                                        int wide_ints) {
-  extern __shared__ __align__(16) int sp_smem[];
+                                                                        int wide_ints, int sc_stride) {
+  extern __shared__ __align__(16) double sp_smem_d[];
   __shared__ unsigned sbm[kSelPlanWarps][2][R];
   __shared__ int ssrc[kSelPlanWarps][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -160,7 +162,20 @@ __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectA
   if (u >= se.U) return;
   const int C = pl.C;
   const bool reg_plan = offloaded && C <= 32 && pl.k <= 32;
+  double* s_sc = sp_smem_d + (size_t)warp * sc_stride;
+  int* sp_smem = reinterpret_cast<int*>(sp_smem_d + (size_t)kSelPlanWarps * sc_stride);
   int* s_sel = sp_smem + (size_t)warp * wide_ints;
+  {
+    // the unit's closed blocks' scores, in a copy group of their own
+    const int n = se.ds->n_closed;
+    const double* g_sc = se.scores + (size_t)u * se.max_blocks;
+    if ((reinterpret_cast<uintptr_t>(g_sc) & 15) == 0 && (se.max_blocks & 1) == 0) {
+      for (int c = lane; c < (n + 1) / 2; c += 32) cp_async16(s_sc + 2 * c, g_sc + 2 * c);
+    } else {
+      for (int j = lane; j < n; j += 32) cp_async8(s_sc + j, g_sc + j);
+    }
+    cp_async_commit();
+  }
   int* s_plan = s_sel + se.k;                 // general plan: slot tables, then its scratch
   int* s_bs = s_plan + 2 * C + 2 * pl.k;      // general plan: block -> slot
   int* s_sb = s_plan;                         // register plan: slot -> block [32]
@@ -173,8 +188,10 @@ __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectA
     if (!reg_plan)
       for (int i = lane; i < pl.max_blocks; i += 32) cp_async4(s_bs + i, pl.block_slot + (size_t)u * pl.max_blocks + i);
   }
-  select_unit_reg<R>(se, u, lane, sbm[warp], se.scores + (size_t)u * se.max_blocks, se.prev + (size_t)u * se.k,
-                     se.ge + (size_t)u * se.k_e, s_sel);
+  cp_async_commit();
+  cp_async_wait_group<1>();  // the scores (the tables may still be on their way)
+  __syncwarp();
+  select_unit_reg<R>(se, u, lane, sbm[warp], s_sc, se.prev + (size_t)u * se.k, se.ge + (size_t)u * se.k_e, s_sel);
   cp_async_wait_all();
   __syncwarp();  // the selection and the tables are read back by the plan
   if (!offloaded) {
@@ -192,7 +209,8 @@ cudaError_t launch_select_plan_r(const SelectArgs& se, const PlanArgs& pl, int o
                                  bool pdl) {
   const bool reg_plan = offloaded && pl.C <= 32 && pl.k <= 32;
   const int wide_ints = se.k + (!offloaded ? 0 : reg_plan ? 64 : 2 * pl.C + 2 * pl.k + pl.max_blocks);
-  const size_t smem = (size_t)kSelPlanWarps * wide_ints * sizeof(int);
+  const int sc_stride = (se.max_blocks + 1) & ~1;
+  const size_t smem = (size_t)kSelPlanWarps * (sc_stride * sizeof(double) + wide_ints * sizeof(int));
   if (smem > 48 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(select_plan_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -200,7 +218,7 @@ cudaError_t launch_select_plan_r(const SelectArgs& se, const PlanArgs& pl, int o
   }
   const int grid = (se.U + kSelPlanWarps - 1) / kSelPlanWarps;
   return launch_ex(select_plan_kernel<R>, dim3(grid), dim3(kSelPlanWarps * 32), smem, st, pdl, 0, se, pl, offloaded,
-                   wide_ints);
+                   wide_ints, sc_stride);
 }
 
 bool select_plan_supported(int max_blocks) { return max_blocks <= 1024; }

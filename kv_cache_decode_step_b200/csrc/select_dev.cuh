@@ -105,23 +105,43 @@ __device__ __forceinline__ void keep_best_reg(uint32_t& mask, int c, const unsig
 
 // Blocks of the per-lane masks, ascending, into out[0..cap) and, when given,
 // into out2 and out3 as well (one walk over the rows); returns the count.
+// Up to 8 rows per lane all R ballots are taken first (they do not depend on
+// one another) and the positions follow from their running counts; with more
+// rows, one row at a time (fewer registers live).
 template <int R>
 __device__ __forceinline__ int write_list_reg(uint32_t mask, int* out, int cap, int lane, int* out2 = nullptr,
                                               int* out3 = nullptr) {
   const unsigned lt = (1u << lane) - 1u;
   int base = 0;
-#pragma unroll 4
-  for (int i = 0; i < R; ++i) {
-    const bool on = (mask >> i) & 1u;
-    const unsigned bal = __ballot_sync(kFull, on);
-    const int pos = base + __popc(bal & lt);
-    if (on && pos < cap) {
-      const int j = 32 * i + lane;
-      out[pos] = j;
-      if (out2) out2[pos] = j;
-      if (out3) out3[pos] = j;
+  if constexpr (R <= 8) {
+    unsigned bal[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) bal[i] = __ballot_sync(kFull, (mask >> i) & 1u);
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int pos = base + __popc(bal[i] & lt);
+      if (((mask >> i) & 1u) && pos < cap) {
+        const int j = 32 * i + lane;
+        out[pos] = j;
+        if (out2) out2[pos] = j;
+        if (out3) out3[pos] = j;
+      }
+      base += __popc(bal[i]);
     }
-    base += __popc(bal);
+  } else {
+#pragma unroll 4
+    for (int i = 0; i < R; ++i) {
+      const bool on = (mask >> i) & 1u;
+      const unsigned bal = __ballot_sync(kFull, on);
+      const int pos = base + __popc(bal & lt);
+      if (on && pos < cap) {
+        const int j = 32 * i + lane;
+        out[pos] = j;
+        if (out2) out2[pos] = j;
+        if (out3) out3[pos] = j;
+      }
+      base += __popc(bal);
+    }
   }
   return base;
 }
