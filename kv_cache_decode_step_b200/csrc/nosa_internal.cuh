@@ -106,7 +106,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
-// 2-D tiled TMA load (no multicast) of one box into shared memory, completing
+// 2-D tiled TMA load of one box into this CTA's shared memory only, completing
 // on an mbarrier.  x is the innermost coordinate (elements), y the row.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
                                             int y) {
@@ -143,7 +143,7 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
                : "memory");
 }
 
-// Untiled bulk copy global -> shared (no multicast), completing on an
+// Untiled bulk copy global -> this CTA's shared memory, completing on an
 // mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
