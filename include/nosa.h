@@ -122,7 +122,18 @@ typedef struct {
  * pooled keys bf16 [U, max_blocks*R, d], agnostic scores fp32 [U, max_blocks],
  * selection state, the GPU block cache bf16 [U, cache_slots, P, d] x 2 (K, V)
  * with its tables, the open tail block bf16 [U, P, d] x 2 and attention
- * partials.  Synchronous.  *out is set only on NOSA_OK. */
+ * partials.  Synchronous.  *out is set only on NOSA_OK.
+ *
+ * Launch shapes are sized from the device's SM count and may be overridden by
+ * environment variables read here, once per context; none of them changes a
+ * result bit: NOSA_GATHER_CTAS (gather CTAs), NOSA_ATTN_CTAS, NOSA_ATTN_STAGES
+ * (2 or 3), NOSA_ATTN_GAP (0..64 empty positions per unit) and
+ * NOSA_ATTN_PRODUCER=0 (hits pass without its producer warp),
+ * NOSA_KV_EVICT_FIRST=0 (hits-pass K/V loads without the L2 evict-first
+ * policy), NOSA_PDL=0 (gather not launched as a programmatic dependent of the
+ * plan), NOSA_PLACED_WIDEN=0 (scoring widens every key by conversion) and
+ * NOSA_WARM_BLOCKS (0..64, default 12: KV in HBM, blocks per hits-pass CTA
+ * prefetched into L2 during the selection). */
 NOSA_API nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out);
 
 /* Free everything nosa_create allocated (synchronises the device first).
