@@ -125,15 +125,17 @@ typedef struct {
  * partials.  Synchronous.  *out is set only on NOSA_OK.
  *
  * Launch shapes are sized from the device's SM count and may be overridden by
- * environment variables read here, once per context; none of them changes a
- * result bit: NOSA_GATHER_CTAS (gather CTAs), NOSA_ATTN_CTAS, NOSA_ATTN_STAGES
- * (2 or 3), NOSA_ATTN_GAP (0..64 empty positions per unit) and
- * NOSA_ATTN_PRODUCER=0 (hits pass without its producer warp),
- * NOSA_KV_EVICT_FIRST=0 (hits-pass K/V loads without the L2 evict-first
- * policy), NOSA_PDL=0 (gather not launched as a programmatic dependent of the
- * plan), NOSA_PLACED_WIDEN=0 (scoring widens every key by conversion) and
- * NOSA_WARM_BLOCKS (0..64, default 12: KV in HBM, blocks per hits-pass CTA
- * prefetched into L2 during the selection). */
+ * environment variables read here, once per context.  None changes a score,
+ * selection, fetch list or cache map.  These change no bit of the output
+ * either: NOSA_GATHER_CTAS (gather CTAs), NOSA_ATTN_PRODUCER=0 (hits pass
+ * without its producer warp), NOSA_KV_EVICT_FIRST=0 (hits-pass K/V loads
+ * without the L2 evict-first policy), NOSA_PDL=0 (gather not launched as a
+ * programmatic dependent of the plan), NOSA_PLACED_WIDEN=0 (scoring widens
+ * every key by conversion) and NOSA_WARM_BLOCKS (0..64, default 12: KV in HBM,
+ * blocks per hits-pass CTA prefetched into L2 during the selection).
+ * NOSA_ATTN_CTAS, NOSA_ATTN_STAGES (2 or 3) and NOSA_ATTN_GAP (0..64 empty
+ * positions per unit) change the hits pass's split of each unit into partial
+ * sums, so outputs may differ from the default in their last bits. */
 NOSA_API nosa_status nosa_create(const nosa_config* cfg, nosa_ctx** out);
 
 /* Free everything nosa_create allocated (synchronises the device first).
