@@ -135,44 +135,45 @@ cudaError_t launch_prepare_r(PrepareArgs a, cudaStream_t st) {
 bool prepare_supported(int max_blocks) { return max_blocks <= kPrepareMaxBlocks; }
 
 // Beyond kPrepareMaxBlocks the scores come from score_kernel (many CTAs per
-// unit); selection and plan then still run as one launch: one warp per unit
-// selects (register path, up to 1024 blocks) and plans from a copy of the
-// selection in shared memory.  The unit's slot tables (and, for the general
-// plan, its block -> slot table) arrive in shared memory by cp.async while
-// the selection runs, so the plan reads no global memory of its own.
-// Shared memory: each warp's copy of its unit's scores [sc_stride] fp64 (read
-// from global memory in one burst of 16-byte copies rather than one load per
-// block and lane), then per warp (wide_ints): the selection [k], then the
-// general plan's scratch (2C + 2k ints, slot tables first) and block -> slot
-// table [max_blocks], or the register plan's slot tables [32] x 2.
+// unit); selection and plan then still run as one launch, one CTA per unit:
+// its kSelPlanWarps warps select together (the group path of select_dev.cuh,
+// 8 or 4 rows of the unit's up to 1024 blocks per lane), then warp 0 plans
+// from a copy of the selection in shared memory.  The unit's scores arrive in
+// shared memory in one burst of 16-byte copies before the selection reads
+// them; its slot tables (and, for the general plan, its block -> slot table)
+// arrive by cp.async while the selection runs, so the plan reads no global
+// memory of its own.  Shared memory: the scores [sc_stride] fp64, then
+// (wide_ints) the selection [k], then the general plan's scratch (2C + 2k
+// ints, slot tables first) and block -> slot table [max_blocks], or the
+// register plan's slot tables [32] x 2.
 constexpr int kSelPlanWarps = 4;
 
 template <int R>
 __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectArgs se, PlanArgs pl, int offloaded,
                                                                         int wide_ints, int sc_stride) {
+  constexpr int RW = R / kSelPlanWarps;
   extern __shared__ __align__(16) double sp_smem_d[];
-  __shared__ unsigned sbm[kSelPlanWarps][2][R];
-  __shared__ int ssrc[kSelPlanWarps][32];
+  __shared__ unsigned sbm[2 * R];
+  __shared__ unsigned red[2 * kSelPlanWarps * 4];
+  __shared__ int ssrc[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u = blockIdx.x * kSelPlanWarps + warp;
+  const int u = blockIdx.x;
   grid_dep_wait();    // the scores are complete
   grid_dep_launch();  // the gather that follows may be placed
   // the gather that follows claims its entries from 0
   if (blockIdx.x == 0 && threadIdx.x == 0) se.ds->gather_next = 0;
-  if (u >= se.U) return;
   const int C = pl.C;
   const bool reg_plan = offloaded && C <= 32 && pl.k <= 32;
-  double* s_sc = sp_smem_d + (size_t)warp * sc_stride;
-  int* sp_smem = reinterpret_cast<int*>(sp_smem_d + (size_t)kSelPlanWarps * sc_stride);
-  int* s_sel = sp_smem + (size_t)warp * wide_ints;
+  double* s_sc = sp_smem_d;
+  int* s_sel = reinterpret_cast<int*>(sp_smem_d + sc_stride);
   {
     // the unit's closed blocks' scores, in a copy group of their own
     const int n = se.ds->n_closed;
     const double* g_sc = se.scores + (size_t)u * se.max_blocks;
     if ((reinterpret_cast<uintptr_t>(g_sc) & 15) == 0 && (se.max_blocks & 1) == 0) {
-      for (int c = lane; c < (n + 1) / 2; c += 32) cp_async16(s_sc + 2 * c, g_sc + 2 * c);
+      for (int c = threadIdx.x; c < (n + 1) / 2; c += blockDim.x) cp_async16(s_sc + 2 * c, g_sc + 2 * c);
     } else {
-      for (int j = lane; j < n; j += 32) cp_async8(s_sc + j, g_sc + j);
+      for (int j = threadIdx.x; j < n; j += blockDim.x) cp_async8(s_sc + j, g_sc + j);
     }
     cp_async_commit();
   }
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectA
   int* s_bs = s_plan + 2 * C + 2 * pl.k;      // general plan: block -> slot
   int* s_sb = s_plan;                         // register plan: slot -> block [32]
   int* s_lu = s_plan + 32;                    //                slot -> last step [32]
-  if (offloaded) {
+  if (offloaded && warp == 0) {
     for (int i = lane; i < C; i += 32) {
       cp_async4(s_sb + i, pl.slot_block + (size_t)u * C + i);
       cp_async4((reg_plan ? s_lu : s_plan + C) + i, pl.last_used + (size_t)u * C + i);
@@ -189,16 +190,19 @@ __global__ void __launch_bounds__(kSelPlanWarps * 32) select_plan_kernel(SelectA
       for (int i = lane; i < pl.max_blocks; i += 32) cp_async4(s_bs + i, pl.block_slot + (size_t)u * pl.max_blocks + i);
   }
   cp_async_commit();
-  cp_async_wait_group<1>();  // the scores (the tables may still be on their way)
-  __syncwarp();
-  select_unit_reg<R>(se, u, lane, sbm[warp], s_sc, se.prev + (size_t)u * se.k, se.ge + (size_t)u * se.k_e, s_sel);
+  cp_async_wait_group<1>();  // this thread's score copies (the tables may still be on their way)
+  __syncthreads();           // and everyone else's
+  SelGroup<kSelPlanWarps> g{red, warp, lane, 1};
+  select_unit_group<RW, kSelPlanWarps>(se, u, g, sbm, s_sc, se.prev + (size_t)u * se.k, se.ge + (size_t)u * se.k_e,
+                                       s_sel);
   cp_async_wait_all();
-  __syncwarp();  // the selection and the tables are read back by the plan
+  __syncthreads();  // the selection and the tables are read back by the plan
+  if (warp != 0) return;
   if (!offloaded) {
     for (int i = lane; i < se.k; i += 32) pl.fetch[(size_t)u * se.k + i] = -1;
     if (lane == 0) pl.n_fetch[u] = 0;
   } else if (reg_plan) {
-    plan_unit_reg(pl, u, lane, ssrc[warp], s_sel, s_sb, s_lu);
+    plan_unit_reg(pl, u, lane, ssrc, s_sel, s_sb, s_lu);
   } else {
     plan_unit_smem(pl, u, lane, s_plan, s_sel, s_bs, true);
   }
@@ -210,14 +214,13 @@ cudaError_t launch_select_plan_r(const SelectArgs& se, const PlanArgs& pl, int o
   const bool reg_plan = offloaded && pl.C <= 32 && pl.k <= 32;
   const int wide_ints = se.k + (!offloaded ? 0 : reg_plan ? 64 : 2 * pl.C + 2 * pl.k + pl.max_blocks);
   const int sc_stride = (se.max_blocks + 1) & ~1;
-  const size_t smem = (size_t)kSelPlanWarps * (sc_stride * sizeof(double) + wide_ints * sizeof(int));
+  const size_t smem = sc_stride * sizeof(double) + (size_t)wide_ints * sizeof(int);
   if (smem > 48 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(select_plan_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  const int grid = (se.U + kSelPlanWarps - 1) / kSelPlanWarps;
-  return launch_ex(select_plan_kernel<R>, dim3(grid), dim3(kSelPlanWarps * 32), smem, st, pdl, 0, se, pl, offloaded,
+  return launch_ex(select_plan_kernel<R>, dim3(se.U), dim3(kSelPlanWarps * 32), smem, st, pdl, 0, se, pl, offloaded,
                    wide_ints, sc_stride);
 }
 
