@@ -7,9 +7,10 @@
 // replacement mapping).  The arithmetic is that of score_kernel,
 // select_reg_kernel and the planning kernels: the same device functions run
 // here, only the launch boundaries between them are gone.  One CTA owns one
-// unit: its four warps score every closed block (scores kept in shared
-// memory), then warp 0 selects and plans.  The gather can start as soon as
-// this single launch ends instead of after three launches in a row.
+// unit: its 4, 8 or 16 warps score every closed block (scores kept in shared
+// memory), then warp 0 selects and plans while, with KV in HBM, warp 1 warms
+// L2 for the hits pass.  The gather can start as soon as this single launch
+// ends instead of after three launches in a row.
 #include "plan_dev.cuh"
 #include "score_dev.cuh"
 #include "select_dev.cuh"
@@ -18,13 +19,6 @@ namespace nosa {
 
 constexpr int kPrepMaxThreads = 512;
 
-// Shared memory: the unit's query rows [G][16] uint4 (staged when they are
-// read from host memory), scores [max_blocks] fp64, selection bitmaps [2][R] words,
-// plan scratch (max(32, 2C + 2k) ints), then copies of the unit's S(t-1) [k],
-// Gamma_e(t-1) [k_e], the new selection [k], the register plan's slot tables
-// [32] x 2 and the general plan's block -> slot table [max_blocks].  The
-// copies are loaded while the scores stream in, so selection and planning
-// read no global memory of their own.
 // Warp-wide: L2 prefetches of the first warm_blocks positions of every
 // hits-pass CTA whose range starts in unit u, with the block ids of S(t-1)
 // (prev: the unit's copy in shared memory).  The hits pass walks positions
@@ -53,6 +47,13 @@ __device__ __forceinline__ void warm_first_blocks(const PrepareArgs& a, int u, i
   }
 }
 
+// Shared memory: the unit's query rows [G][16] uint4 (staged when they are
+// read from host memory), scores [max_blocks] fp64, selection bitmaps [2][R] words,
+// plan scratch (max(32, 2C + 2k) ints), then copies of the unit's S(t-1) [k],
+// Gamma_e(t-1) [k_e], the new selection [k], the register plan's slot tables
+// [32] x 2 and the general plan's block -> slot table [max_blocks].  The
+// copies are loaded while the scores stream in, so selection and planning
+// read no global memory of their own.
 template <int R>
 __global__ void __launch_bounds__(kPrepMaxThreads, 1) prepare_kernel(PrepareArgs a) {
   extern __shared__ __align__(16) unsigned char prep_smem[];
