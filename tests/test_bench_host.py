@@ -55,3 +55,21 @@ def test_algorithmic_hbm_bytes_of_the_metric_workload(bench):
     U, n, k, F = 512, 64, 16, 500
     want = U * n * 4 * 128 * 2 + U * n * 20 + U * k * 64 * 128 * 4 + F * 64 * 128 * 4 + 64 * 32 * 128 * 4
     assert bench.hbm_bytes_per_step(w, F) == want
+
+
+def test_captured_traffic_is_consistent_with_the_work(bench):
+    """The ncu counters the bench line carries: the gather's link bytes exceed
+    its host-memory payload only by the completions' protocol overhead, and
+    its payload is at most every selected block missing (32 KiB of K and V
+    each); the hits
+    pass reads no more DRAM bytes per launch than the K/V of every selected
+    block of the resident 8B layer (the rest is in L2 when the launch starts)."""
+    ga = bench.NCU_TRAFFIC[("gather_attend_kernel", "offload_b64")]
+    wb = configs.get("offload_b64")
+    assert 0 < ga["payload"] <= wb.units * wb.k * 32 * 1024
+    assert 1.0 < ga["pcie_read"] / ga["payload"] < 1.15
+    assert ga["dram"] < 0.05 * ga["payload"]  # the cache writes stay in L2 during the launch
+    w = configs.get("layer8b")
+    kv_bytes = w.units * w.k * w.block * w.head_dim * 2 * 2
+    hits = bench.NCU_TRAFFIC[("attend_hits_ws_kernel", "layer8b")]
+    assert 0.9 * kv_bytes < hits["dram"] <= kv_bytes
