@@ -426,11 +426,20 @@ def run_ours(args):
 
     # kernels per step: score, select, [plan, gather + miss attention], hits
     # pass -- the fused entry point makes score, select and plan one kernel up
-    # to 512 blocks per unit; with appends also append, close and advance
-    # (otherwise the last unit merged ends the step), and with KV in host
-    # memory the write-through of a block the previous step closed
-    fused = dec.fused and w.max_blocks <= 512
-    launches_per_step = ((3 if w.offloaded else 2) if fused else (5 if w.offloaded else 3)) \
+    # to 512 blocks per unit and two (the scoring grid, then select + plan) up
+    # to 1024; with appends also append, close and advance (otherwise the last
+    # unit merged ends the step), and with KV in host memory the write-through
+    # of a block the previous step closed
+    if dec.fused and w.max_blocks <= 512:
+        first_half, calls = 1, "nosa_score_select_fetch (one kernel) + nosa_sparse_decode"
+    elif dec.fused and w.max_blocks <= 1024:
+        first_half = 2
+        calls = "nosa_score_select_fetch (scoring grid + select/plan kernel) + nosa_sparse_decode"
+    else:
+        # beyond 1024 blocks nosa_score_select_fetch makes these three calls itself
+        first_half = 3 if w.offloaded else 2
+        calls = "nosa_score_blocks + nosa_select + nosa_fetch_missing + nosa_sparse_decode"
+    launches_per_step = first_half + (2 if w.offloaded else 1) \
         + (3 if w.append else 0) + (1 if w.append and w.offloaded else 0)
     gather_ms = phase["gather_ms"]
     attn_ms = phase["attention_ms"]
@@ -481,8 +490,7 @@ def run_ours(args):
             "config": workload_config(base, args.policy, world),
             "run": {"graph": "cuda graph replay",
                     "cpu_affinity": (f"{numa_cpus} CPUs local to the GPU" if numa_cpus else "unchanged"),
-                    "calls": ("nosa_score_select_fetch (fused) + nosa_sparse_decode" if fused
-                              else "nosa_score_blocks + nosa_select + nosa_fetch_missing + nosa_sparse_decode"),
+                    "calls": calls,
                     "hbm_bytes_per_step": hbm_bytes},
             "roofline": dominant,
             "roofline_other": other,
