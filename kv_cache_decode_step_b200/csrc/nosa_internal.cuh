@@ -128,8 +128,8 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
 }
 
 // An L2 policy that makes the lines a load brings in the first to go: for
-// data read once per step (the selected K/V), so that data reused across
-// steps (the pooled keys) stays in L2.
+// data read once per step (the selected K/V), so that it does not push out
+// data reused across steps (the pooled keys) first.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
